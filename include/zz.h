@@ -1,0 +1,188 @@
+/*
+ * libzz — zigzag context-parallel prefill attention for NVIDIA B200 (sm_100a).
+ *
+ * The method (page "sgl-project--sglang/python/sglang/srt/layers/cp/zigzag.py",
+ * module docstring): with cp_size c every sequence is cut into 2c blocks; rank r
+ * owns block r (its "prev" half) and block 2c-1-r (its "next" half).  K/V are
+ * all-gathered in rank order, reranged back to token order and written into a
+ * paged KV pool; then each rank's two query halves run causal attention against
+ * the K/V prefix that ends at their own block.  On one GPU all c ranks are
+ * "virtual" and are computed by one launch.
+ *
+ * Conventions for every entry point:
+ *   - Returns zz_status_t; zz_last_error() gives a thread-local message for the
+ *     last failing call on this thread.  No C++ exception crosses the ABI.
+ *   - The caller owns every device buffer (inputs, outputs, workspace).  The
+ *     library owns only the opaque host-side plan object.
+ *   - Kernel entry points allocate no device memory, do not synchronise the
+ *     host, and enqueue all work on the caller's stream (a cudaStream_t passed
+ *     as void*; NULL means the legacy default stream).
+ *   - Device pointers must be 16-byte aligned.  Integer tables are int32 unless
+ *     stated; pool slot indices are int64.
+ *   - bf16 is IEEE binary16-brain (1-8-7); fp32 is IEEE binary32.
+ */
+#ifndef ZZ_H_
+#define ZZ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ZZ_OK = 0,
+  ZZ_ERR_INVALID_ARG = 1,      /* null/misaligned pointer, bad size, h_q % h_kv != 0, ... */
+  ZZ_ERR_NOT_APPLICABLE = 2,   /* zigzag CP refuses the batch (zigzag.py, can_apply)      */
+  ZZ_ERR_UNSUPPORTED = 3,      /* valid request this build does not implement (d, dtype)  */
+  ZZ_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed                        */
+  ZZ_ERR_DEVICE_TIMEOUT = 5    /* a bounded device-side wait gave up (see zz_attn_status) */
+} zz_status_t;
+
+typedef enum { ZZ_BF16 = 0, ZZ_FP32 = 1 } zz_dtype_t;
+
+typedef struct zz_plan zz_plan_t;
+
+/* Lists of zigzag.py ZigzagContextParallelMetadata, plus derived tables. */
+typedef enum {
+  ZZ_FIELD_EXTEND_LENS = 0,        /* [bs]      extend lengths after the pad fold-in          */
+  ZZ_FIELD_PREFIX = 1,             /* [bs]      cached-prefix tokens per sequence             */
+  ZZ_FIELD_SPLIT_LIST = 2,         /* [bs*2c]   block sizes, sequence-major                    */
+  ZZ_FIELD_ZIGZAG_INDEX = 3,       /* [2*bs]    per rank: prev chunks then next chunks         */
+  ZZ_FIELD_CP_REVERSE_INDEX = 4,   /* [bs*2c]   gathered chunk -> natural order                */
+  ZZ_FIELD_REVERSE_SPLIT_LEN = 5,  /* [c*2*bs]  chunk sizes of the gathered buffer             */
+  ZZ_FIELD_PER_RANK_TOKENS = 6,    /* [c]       per_rank_actual_token                          */
+  ZZ_FIELD_MAX_RANK_LEN = 7,       /* [c]       max_rank_len (all equal, M)                    */
+  ZZ_FIELD_KV_LEN_PREV = 8,        /* [bs]      per rank                                       */
+  ZZ_FIELD_KV_LEN_NEXT = 9,        /* [bs]      per rank                                       */
+  ZZ_FIELD_Q_LEN_PREV = 10,        /* [bs]      per rank (actual_seq_q_prev)                   */
+  ZZ_FIELD_Q_LEN_NEXT = 11,        /* [bs]      per rank (actual_seq_q_next)                   */
+  ZZ_FIELD_CU_SEQLENS_Q_PREV = 12, /* [bs+1]    per rank, local exclusive prefix sums          */
+  ZZ_FIELD_CU_SEQLENS_Q_NEXT = 13, /* [bs+1]    per rank                                       */
+  ZZ_FIELD_SRC_ROW = 14            /* [T]       natural token -> row of the [c*M] layout       */
+} zz_field_t;
+
+typedef struct {
+  int32_t cp_size;
+  int32_t bs;
+  int64_t total_tokens;     /* T = sum of extend lengths after the pad fold-in        */
+  int32_t max_rank_len;     /* M: rows per rank in the padded gathered / Q layouts    */
+  int32_t total_q_prev;     /* of the rank asked for in zz_plan_info                  */
+  int32_t total_q_next;
+  int32_t max_seqlen_q_prev;
+  int32_t max_seqlen_q_next;
+  int64_t causal_pairs;     /* visible (q,k) pairs over all ranks and halves          */
+} zz_plan_info_t;
+
+/* Thread-local message of the last failing call on this thread ("" if none). */
+const char* zz_last_error(void);
+
+/*
+ * Build the zigzag metadata for ALL c ranks on the host
+ * (zigzag.py, ZigzagCPStrategy.can_apply and build_metadata).
+ *   extend_lens [bs]  tokens to prefill per sequence; may be NULL (then
+ *                     seq_lens is used, or one sequence of num_tokens, bs = 1).
+ *   seq_lens    [bs]  total lengths incl. cached prefix; may be NULL (prefix 0).
+ *   num_tokens        >= sum(extend_lens); the surplus is folded into the last
+ *                     sequence (and into seq_lens[bs-1] when given).
+ * Errors: ZZ_ERR_NOT_APPLICABLE if cp_size <= 1, num_tokens < 2c or any extend
+ * length < 2c; ZZ_ERR_INVALID_ARG for bs <= 0, negative lengths, num_tokens <
+ * sum(extend_lens), or sizes beyond int32 rows.  *out is owned by the caller and
+ * released with zz_plan_destroy.  Host only; needs no GPU.
+ */
+zz_status_t zz_plan_create(int cp_size, int bs, const int32_t* extend_lens,
+                           const int32_t* seq_lens, int64_t num_tokens, zz_plan_t** out);
+void zz_plan_destroy(zz_plan_t* plan);
+
+/* Scalars of the plan; the per-rank ones are for `rank`. */
+zz_status_t zz_plan_info(const zz_plan_t* plan, int rank, zz_plan_info_t* out);
+
+/*
+ * Copy one list into host memory.  `rank` selects the rank for per-rank
+ * fields and is ignored otherwise.  On success *count is the list length;
+ * with dst == NULL only *count is written.  ZZ_ERR_INVALID_ARG if capacity is
+ * too small or rank is out of range.
+ */
+zz_status_t zz_plan_get(const zz_plan_t* plan, int rank, zz_field_t field,
+                        int32_t* dst, int64_t capacity, int64_t* count);
+
+/* Bytes of device workspace zz_plan_upload needs (256-byte aligned sections). */
+size_t zz_plan_workspace_bytes(const zz_plan_t* plan);
+
+/*
+ * Enqueue the host-to-device copy of the plan's device tables (token -> row
+ * map, half descriptors, longest-first work lists) into `dev_workspace`
+ * (caller-owned, >= zz_plan_workspace_bytes, 256-byte aligned) on `stream`,
+ * and remember that address for later calls.  The plan must outlive the copy.
+ */
+zz_status_t zz_plan_upload(zz_plan_t* plan, void* dev_workspace, size_t bytes, void* stream);
+
+/*
+ * Read (and optionally clear) the device status word that the kernels of this
+ * plan set when a bounded device-side wait gives up instead of hanging.
+ * Synchronises `stream` (a diagnostic, not a hot-path call).  Returns
+ * ZZ_ERR_DEVICE_TIMEOUT when bit 0 of *flags is set, ZZ_OK otherwise.
+ */
+zz_status_t zz_plan_device_status(const zz_plan_t* plan, int32_t* flags, int clear, void* stream);
+
+/*
+ * Shard rows from natural token order into the rank-ordered padded layout
+ * [c*M, row_bytes] (zigzag.py, shard_hidden_states for every rank, stacked as
+ * _all_gather_reorganized would deliver them).  Padding rows are not written.
+ * src: [T, row_bytes], dst: [c*M, row_bytes]; row_bytes a multiple of 16.
+ */
+zz_status_t zz_shard_rows(const zz_plan_t* plan, const void* src, void* dst,
+                          int64_t row_bytes, void* stream);
+
+/*
+ * Rerange the all-gathered K and V into the paged pool, in one pass
+ * (zigzag.py, _all_gather_reorganized trim + gather_kv_cache + the
+ * set_kv_buffer of materialize_full_kv, with unit k/v scales):
+ *     k_pool[out_cache_loc[t]] = k_gathered[src_row[t]]  for every token t,
+ * and the same for V.
+ *   k_gathered, v_gathered: [c*M, h_kv, d] rank-ordered, padded to M per rank.
+ *   k_pool, v_pool:         [num_slots, h_kv, d].
+ *   out_cache_loc:          [T] int64 pool slots in natural token order.
+ * v_gathered and v_pool may both be NULL (one tensor only).  Slots outside
+ * [0, num_slots) are skipped, never written.  Bit-exact copy: any dtype whose
+ * row h_kv*d*sizeof(dtype) is a multiple of 16 bytes.
+ */
+zz_status_t zz_rerange_kv_to_pool(const zz_plan_t* plan, const void* k_gathered,
+                                  const void* v_gathered, void* k_pool, void* v_pool,
+                                  const int64_t* out_cache_loc, int64_t num_slots,
+                                  int h_kv, int d, zz_dtype_t dtype, void* stream);
+
+/*
+ * Zigzag prefill attention for ranks [rank_begin, rank_begin + rank_count)
+ * in ONE launch (zigzag.py, run_attention: prev half then next half).  For
+ * every rank r, half h, sequence s and query head i:
+ *     O = softmax(scale * Q K^T + causal mask) V
+ * over keys [0, kv_len_h[s]), query row j of the half sitting at position
+ * kv_len_h[s] - Lq + j and seeing keys <= that position; K/V head = i / (h_q/h_kv).
+ *   q, out: [rank_count, M, h_q, d] rank-local rows (prev halves from row 0,
+ *           next halves from row total_q_prev of that rank); padding rows are
+ *           neither read for any valid output nor written.
+ *   k_pool, v_pool: [num_slots, h_kv, d]; page_table [bs, max_pages] int32;
+ *           slot of key t of sequence s = page_table[s][t/page_size]*page_size
+ *           + t%page_size.  Only the first ceil(kv_len/page_size) entries of a
+ *           row are read.
+ *   lse: optional [rank_count, M, h_q] fp32 natural-log sum of exponentials.
+ *   softmax_scale <= 0 selects 1/sqrt(d).
+ * Errors: ZZ_ERR_INVALID_ARG when h_q % h_kv != 0 (message names "multiple of
+ * num_kv_heads"), null or misaligned pointers, rank range outside [0,c);
+ * ZZ_ERR_UNSUPPORTED for d not in {64,128}, or for bf16 a page_size that is
+ * neither 16, 32, 64 nor a multiple of 128.
+ * bf16 runs the tcgen05/TMEM/TMA kernel (fp32 accumulate and softmax); fp32
+ * runs a CUDA-core kernel in full fp32.
+ */
+zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_count,
+                            const void* q, const void* k_pool, const void* v_pool,
+                            int64_t num_slots, const int32_t* page_table, int max_pages,
+                            int page_size, void* out, float* lse, int h_q, int h_kv, int d,
+                            float softmax_scale, zz_dtype_t dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ZZ_H_ */

@@ -1,0 +1,110 @@
+"""Attention parity with the fp64 oracle (GPU), through the C ABI.
+
+Small cases are compared on every valid output row; the full-size
+configurations on sampled rows (first, last and random rows of every half of
+every rank).  Tolerances: bf16 max-abs 2e-2 and mean-abs 2e-3, fp32 max-abs 1e-4.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import rerange as OR
+from tests.gpu_cases import Case, Run, assert_close, zz
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_full(run: Run):
+    run.attend()
+    p = run.ref_plan
+    out = run.out.float().cpu().numpy()
+    lse = run.lse.cpu().numpy()
+    for r in range(p.cp_size):
+        o_ref, l_ref = run.expected_rank(r)
+        n = p.per_rank_actual_token[r]
+        got = out[r * p.M: r * p.M + n]
+        assert np.isfinite(got).all()
+        assert_close(got, o_ref, run.case.dtype, f"rank {r} out")
+        assert np.abs(lse[r * p.M: r * p.M + n] - l_ref).max() < 2e-3, f"rank {r} lse"
+
+
+SMALL = [
+    Case(2, [256], 4, 4, 64, dtype="fp32", page_size=256, scale=1.0, page_seed=None),  # fp32, unpaged
+    Case(2, [300, 517], 8, 2, 128, page_size=16),          # GQA 4, ragged blocks and tails
+    Case(3, [700], 4, 4, 128, page_size=64),               # MHA: row-tile pairs
+    Case(2, [333], 6, 2, 128, page_size=32),               # odd group (3)
+    Case(2, [600, 129], 8, 1, 128, page_size=16),          # MQA
+    Case(2, [400], 4, 2, 64, page_size=32),                # bf16 head_dim 64
+    Case(2, [1000], 4, 2, 128, page_size=256),             # page larger than a K/V tile
+    Case(4, [1100, 600], 4, 2, 128, page_size=8),          # page 8
+    Case(2, [260, 300], 4, 2, 128, page_size=16, prefix=[100, 37]),   # cached prefix
+    Case(2, [96], 2, 1, 128, page_size=16),                # every half shorter than one tile
+    Case(2, [48], 2, 2, 64, dtype="fp32", page_size=16),   # fp32 paged
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"c{c.cp}-L{c.lens}-{c.h_q}/{c.h_kv}-d{c.d}-{c.dtype}-ps{c.page_size}")
+def test_small_cases_every_row(case):
+    _check_full(Run(case))
+
+
+def test_c4_L4096_gqa8_every_row():
+    _check_full(Run(Case(4, [4096], 32, 4, 128, page_size=16)))
+
+
+def test_single_rank_launches_match_full_launch():
+    run = Run(Case(4, [1500, 700], 8, 2, 128, page_size=16))
+    run.attend()
+    full = run.out.clone()
+    p = run.ref_plan
+    for r in range(p.cp_size):
+        run.out.fill_(float("nan"))
+        q_r = run.q_ranked[r * p.M:(r + 1) * p.M]
+        out_r = torch.full_like(q_r, float("nan"))
+        zz.attn_prefill(run.plan, q_r, run.k_pool, run.v_pool, run.page_table, 16, out_r,
+                        softmax_scale=run.softmax_scale, rank_begin=r, rank_count=1)
+        torch.cuda.synchronize()
+        n = p.per_rank_actual_token[r]
+        assert torch.equal(out_r[:n], full[r * p.M: r * p.M + n])
+
+
+def test_union_in_token_order_equals_unsharded_attention():
+    """Outputs of all ranks, moved back to token order, equal plain causal attention."""
+    from oracle import attention as OA
+    run = Run(Case(4, [2000], 8, 2, 128, page_size=16))
+    run.attend()
+    p = run.ref_plan
+    o_tok = OR.gather_kv(run.out.float().cpu().numpy(), p)
+    ref, _ = OA.full_causal(run.q.double().cpu().numpy(), run.k_seqs[0].double().cpu().numpy(),
+                            run.v_seqs[0].double().cpu().numpy(), run.softmax_scale)
+    assert_close(o_tok, ref, "bf16", "union")
+
+
+def _check_sampled(run: Run, per_half: int):
+    run.attend()
+    samples = run.sampled_rows(per_half)
+    want = run.expected_rows(samples)
+    out = run.out
+    lse = run.lse
+    p = run.ref_plan
+    got = np.stack([out[r * p.M + lrow].float().cpu().numpy() for (r, lrow, *_rest) in samples])
+    ref = np.stack([w[0] for w in want])
+    assert np.isfinite(got).all()
+    assert_close(got, ref, "bf16", "sampled rows")
+    gl = np.stack([lse[r * p.M + lrow].cpu().numpy() for (r, lrow, *_rest) in samples])
+    assert np.abs(gl - np.stack([w[1] for w in want])).max() < 2e-3
+
+
+def test_varlen_batch_c4_sampled_rows():
+    lens = synth.varlen_lengths(8, 1000, 8192, seed=0)
+    _check_sampled(Run(Case(4, lens, 32, 4, 128, page_size=16)), per_half=6)
+
+
+@pytest.mark.parametrize("h_q,h_kv,cp", [(32, 32, 2), (32, 8, 4), (32, 1, 8)])
+def test_L32768_head_ratio_sweep_sampled_rows(h_q, h_kv, cp):
+    _check_sampled(Run(Case(cp, [32768], h_q, h_kv, 128, page_size=16)), per_half=3)
+
+
+def test_long_context_c8_L131072_sampled_rows():
+    _check_sampled(Run(Case(8, [131072], 64, 8, 128, page_size=64)), per_half=2)

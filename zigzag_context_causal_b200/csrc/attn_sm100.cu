@@ -1,0 +1,586 @@
+// Zigzag prefill attention on the 5th-generation tensor core (sm_100a).
+//
+// Problem (page "sgl-project--sglang/python/sglang/srt/layers/cp/zigzag.py",
+// run_attention + build_metadata): for every virtual rank r, half h in
+// {prev, next}, sequence s and query head i, causal attention of the half's
+// Lq query rows against the first kv_len keys of the sequence; query row j sits
+// at position kv_len - Lq + j.  Grouped K/V: query head i reads K/V head
+// i / (H_q/H_kv) ("PR #34485 完整报告", implementation item 1).
+//
+// One CTA owns two 128-row query sub-tiles that stream the SAME K/V tiles:
+//   * even GQA group: the same rows of two query heads that share a K/V head
+//     (identical causal extent), or
+//   * otherwise: two consecutive row tiles of one head (the second one sees
+//     one more K/V tile at most).
+// Warp roles (320 threads):
+//   warps 0-3  softmax for sub-tile 0   (thread = TMEM lane = query row)
+//   warps 4-7  softmax for sub-tile 1
+//   warp  8    MMA issue (one thread) + TMEM allocation
+//   warp  9    TMA producer: Q once, then K_j, V_j into a ring of smem slots
+// TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [256+D,256+2D).
+// P (bf16, two per column) overwrites the first 64 columns of its S tile and
+// feeds the P.V MMA straight from TMEM.  The MMA order per K/V tile j is
+//   PV0(j)  S0(j+1)  PV1(j)  S1(j+1)
+// so each softmax group works on one tile while the tensor core runs the
+// other group's MMAs.  The softmax keeps a running maximum in log2 units and
+// only rescales O (in TMEM) when the maximum grows by more than 8, so most
+// tiles skip the correction.  Tiles past the causal diagonal are never loaded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include <mutex>
+#include <string>
+
+#include "ptx_sm100.cuh"
+#include "zz_internal.h"
+
+namespace zz {
+
+zz_status_t launch_attn_simt_fp32(const zz_plan_t* p, int rank_begin, int rank_count,
+                                  const void* q, const void* k_pool, const void* v_pool,
+                                  int64_t num_slots, const int32_t* page_table, int max_pages,
+                                  int page_size, void* out, float* lse, int h_q, int h_kv, int d,
+                                  float scale, cudaStream_t s);
+
+namespace {
+
+using namespace zz::dev;
+
+constexpr int kThreads = 320;
+constexpr int kWarpMma = 8;
+constexpr int kWarpLoad = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 256 between rescales
+
+template <int D>
+struct Cfg {
+  static constexpr int kBoxes = D / 64;                  // 128-byte swizzle boxes per row
+  static constexpr int kBoxBytes = 128 * 128;            // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one Q, K or V tile
+  static constexpr int kSlots = D == 64 ? 8 : 4;         // K/V ring depth
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
+  static constexpr int kSmem = kBarOff + 512 + 1024;     // + barriers + alignment slack
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+};
+
+struct Params {
+  const HalfDesc* halves;
+  const WorkItem* items;
+  const int32_t* page_table;
+  const __nv_bfloat16* k_pool;
+  const __nv_bfloat16* v_pool;
+  __nv_bfloat16* out;
+  float* lse;
+  int* status;
+  int64_t num_slots;
+  int h_q, h_kv, group;
+  int pair_heads;       // 1: sub-tiles are heads 2g, 2g+1; 0: row tiles 2t, 2t+1 of head g
+  int head_groups;      // CTAs per work item
+  int M, rank_begin;
+  int max_pages, page_size, box_rows;
+  float scale_log2;
+  uint64_t timeout_ns;
+};
+
+struct Bars {
+  uint64_t q_full[2];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t mma_done;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct SubTile {
+  int head;
+  int q0;   // first half-local row
+  int n;    // K/V tiles to visit (0 = empty sub-tile)
+};
+
+__device__ __forceinline__ int tiles_for(const HalfDesc& h, int q0) {
+  if (q0 >= h.lq) return 0;
+  const int last_row = min(q0 + 128, h.lq) - 1;
+  return (h.kv_pos0 + last_row) / 128 + 1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::kBarOff);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work decomposition ----
+  const WorkItem w = p.items[blockIdx.x / p.head_groups];
+  const int hg = blockIdx.x % p.head_groups;
+  const HalfDesc hd = p.halves[w.half_id];
+  SubTile st[2];
+  if (p.pair_heads) {
+    st[0] = {2 * hg, w.tile * 128, 0};
+    st[1] = {2 * hg + 1, w.tile * 128, 0};
+  } else {
+    st[0] = {hg, (2 * w.tile) * 128, 0};
+    st[1] = {hg, (2 * w.tile + 1) * 128, 0};
+  }
+  st[0].n = tiles_for(hd, st[0].q0);
+  st[1].n = tiles_for(hd, st[1].q0);
+  const int n_max = max(st[0].n, st[1].n);
+  const int kv_head = st[0].head / p.group;
+  const int64_t row_base = int64_t(hd.rank - p.rank_begin) * p.M + hd.row0;  // Q/O row of half row 0
+
+  // ---- setup ----
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q_full[i], 1);
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_full[i], 1);
+    }
+    mbar_init(&bars->mma_done, 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    // A CTA that timed out earlier in this launch (or an earlier launch of
+    // this plan) has set the status word: skip the work instead of waiting.
+    bars->abort = (p.status && *reinterpret_cast<volatile int*>(p.status)) ? 1 : 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == kWarpLoad) {
+    // ================= TMA producer =================
+    const int32_t* pt = p.page_table + int64_t(hd.seq) * p.max_pages;
+    bool q_issued[2] = {false, false};
+    if (lane == 0 && !*abort) {
+      for (int i = 0; i < 2; ++i) {
+        if (st[i].n == 0) continue;
+        q_issued[i] = true;
+        uint8_t* dst = smem + C::kQOff + i * C::kTileBytes;
+        mbar_arrive_expect_tx(&bars->q_full[i], C::kTileBytes);
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_3d(dst + b * C::kBoxBytes, &tm_q, &bars->q_full[i], b * 64, st[i].head,
+                      int32_t(row_base + st[i].q0));
+      }
+    }
+    int load_no = 0;
+    const int chunks = 128 / p.box_rows;
+    for (int j = 0; j < n_max && !*abort; ++j) {
+      for (int t = 0; t < 2; ++t, ++load_no) {
+        const int slot = load_no % C::kSlots;
+        const uint32_t use = load_no / C::kSlots;
+        if (!wait_parity(&bars->kv_empty[slot], (use & 1u) ^ 1u, abort, p.timeout_ns)) break;
+        uint8_t* tile = smem + C::kKVOff + slot * C::kTileBytes;
+        const __nv_bfloat16* pool = t == 0 ? p.k_pool : p.v_pool;
+        const void* tm = t == 0 ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
+        const int key0 = j * 128;
+        // Rows at or beyond kv_len (end of the sequence's keys) are filled by
+        // hand: real keys copied, the rest zero, so no stale or unwritten pool
+        // slot can reach the MMAs (0 * NaN would poison P.V).
+        uint32_t tma_bytes = 0;
+        bool manual = false;
+        for (int c = 0; c < chunks; ++c) {
+          if (key0 + (c + 1) * p.box_rows <= hd.kv_len) tma_bytes += p.box_rows * 128 * C::kBoxes;
+          else manual = true;
+        }
+        if (manual) {
+          const int units_per_row = C::kBoxes * 8;
+          for (int c = 0; c < chunks; ++c) {
+            if (key0 + (c + 1) * p.box_rows <= hd.kv_len) continue;
+            const int r_lo = c * p.box_rows;
+            for (int u = lane; u < p.box_rows * units_per_row; u += 32) {
+              const int row = r_lo + u / units_per_row;
+              const int rem = u % units_per_row;
+              const int b = rem >> 3, ch = rem & 7;
+              const int key = key0 + row;
+              int4 v = make_int4(0, 0, 0, 0);
+              if (key < hd.kv_len) {
+                const int64_t slot_id = int64_t(__ldg(pt + key / p.page_size)) * p.page_size + key % p.page_size;
+                if (slot_id >= 0 && slot_id < p.num_slots)
+                  v = __ldg(reinterpret_cast<const int4*>(pool + (slot_id * p.h_kv + kv_head) * D + b * 64 + ch * 8));
+              }
+              *reinterpret_cast<int4*>(tile + b * C::kBoxBytes + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars->kv_full[slot], tma_bytes);
+          for (int c = 0; c < chunks; ++c) {
+            const int kc = key0 + c * p.box_rows;
+            if (kc + p.box_rows > hd.kv_len) continue;
+            const int32_t slot0 = __ldg(pt + kc / p.page_size) * p.page_size + kc % p.page_size;
+            for (int b = 0; b < C::kBoxes; ++b)
+              tma_load_3d(tile + b * C::kBoxBytes + c * p.box_rows * 128, tm, &bars->kv_full[slot],
+                          b * 64, kv_head, slot0);
+          }
+        }
+        __syncwarp();
+      }
+    }
+    // Never leave with copies in flight into shared memory.
+    if (lane == 0) {
+      for (int n = max(0, load_no - C::kSlots); n < load_no; ++n)
+        drain_parity(&bars->kv_full[n % C::kSlots], (uint32_t(n / C::kSlots)) & 1u, p.timeout_ns);
+      for (int i = 0; i < 2; ++i)
+        if (q_issued[i]) drain_parity(&bars->q_full[i], 0, p.timeout_ns);
+    }
+  } else if (warp == kWarpMma) {
+    // ================= MMA issue (single thread) =================
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(smem + C::kQOff);
+      const uint32_t kv_addr = smem_u32(smem + C::kKVOff);
+      const uint32_t col_s[2] = {C::kColS0, C::kColS1};
+      const uint32_t col_o[2] = {C::kColO0, C::kColO1};
+      auto slot_of = [](int n) { return n % C::kSlots; };
+      auto par_of = [](int n) { return uint32_t(n / C::kSlots) & 1u; };
+      auto issue_s = [&](int i, int slot) {
+        const uint32_t qa = q_addr + i * C::kTileBytes;
+        const uint32_t ka = kv_addr + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+          mma_ss(tmem + col_s[i], smem_desc_sw128(qa + off, 16, 1024),
+                 smem_desc_sw128(ka + off, 16, 1024), idesc_s, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int i, int slot, bool acc) {
+        const uint32_t va = kv_addr + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(tmem + col_o[i], tmem + col_s[i] + kk * 8,
+                 smem_desc_sw128(va + kk * 2048, C::kBoxBytes, 1024), idesc_o, acc || kk > 0);
+      };
+      bool ok = true;
+      for (int i = 0; i < 2 && ok; ++i)
+        if (st[i].n) ok = wait_parity(&bars->q_full[i], 0, abort, p.timeout_ns);
+      if (ok && n_max > 0) ok = wait_parity(&bars->kv_full[slot_of(0)], par_of(0), abort, p.timeout_ns);
+      if (ok && n_max > 0) {
+        tc_fence_after();
+        for (int i = 0; i < 2; ++i)
+          if (st[i].n) {
+            issue_s(i, slot_of(0));
+            mma_commit(&bars->s_full[i]);
+          }
+        mma_commit(&bars->kv_empty[slot_of(0)]);
+      }
+      for (int j = 0; j < n_max && ok; ++j) {
+        const int nv = 2 * j + 1, nk = 2 * j + 2;
+        if (!(ok = wait_parity(&bars->kv_full[slot_of(nv)], par_of(nv), abort, p.timeout_ns))) break;
+        tc_fence_after();
+        bool k_ready = false;
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (j >= st[i].n) continue;
+          if (!(ok = wait_parity(&bars->p_full[i], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+          tc_fence_after();
+          issue_pv(i, slot_of(nv), j > 0);
+          if (j == st[i].n - 1) mma_commit(&bars->o_full[i]);
+          if (j + 1 < st[i].n) {
+            if (!k_ready) {
+              if (!(ok = wait_parity(&bars->kv_full[slot_of(nk)], par_of(nk), abort, p.timeout_ns))) break;
+              tc_fence_after();
+              k_ready = true;
+            }
+            issue_s(i, slot_of(nk));
+            mma_commit(&bars->s_full[i]);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&bars->kv_empty[slot_of(nv)]);
+        if (j + 1 < n_max) {
+          if (!k_ready) {  // the next K tile is only used by the longer sub-tile
+            if (!(ok = wait_parity(&bars->kv_full[slot_of(nk)], par_of(nk), abort, p.timeout_ns))) break;
+            tc_fence_after();
+          }
+          mma_commit(&bars->kv_empty[slot_of(nk)]);
+        }
+      }
+      // Drain: no MMA may still be running when TMEM is released.
+      mma_commit(&bars->mma_done);
+      drain_parity(&bars->mma_done, 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ================= softmax + epilogue (warps 0-7) =================
+    const int g = warp >> 2;                   // sub-tile
+    const SubTile& me = st[g];
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;         // TMEM lane == row of the sub-tile
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + (g ? C::kColS1 : C::kColS0);
+    const uint32_t t_o = tmem + lane_off + (g ? C::kColO1 : C::kColO0);
+    const int q_row = me.q0 + r;
+    const int my_pos = hd.kv_pos0 + q_row;     // last visible key (inclusive)
+    float m = -CUDART_INF_F, l = 0.f;
+    bool ok = me.n > 0;
+    for (int j = 0; j < me.n && ok; ++j) {
+      if (!(ok = wait_parity(&bars->s_full[g], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+      tc_fence_after();
+      // Pass 1: row maximum over the visible columns (S read 64 columns at a time).
+      const int limit = my_pos - j * 128 + 1;   // visible keys of this tile
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a[32], b[32];
+        tmem_ld32(t_s + h * 64, a);
+        tmem_ld32(t_s + h * 64 + 32, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float x = (h * 64 + e < limit) ? __uint_as_float(a[e]) : -CUDART_INF_F;
+          const float y = (h * 64 + 32 + e < limit) ? __uint_as_float(b[e]) : -CUDART_INF_F;
+          mx = fmaxf(mx, fmaxf(x, y));
+        }
+      }
+      const float m_tile = mx * p.scale_log2;
+      if (j == 0) {
+        m = m_tile;
+      } else if (m_tile > m + kRescaleThreshold) {
+        // S(j) completing implies P.V(j-1) completed: O is stable here.
+        const float f = ex2(m - m_tile);
+        l *= f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+          tmem_st32(t_o + c * 32, o);
+        }
+        m = m_tile;
+      }
+      // Pass 2: P = 2^(s*scale*log2e - m), summed in fp32, packed to bf16 over
+      // the first 64 columns of S.  Columns are re-read before being overwritten.
+      const float neg_m = -m;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(t_s + c * 32, sv);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int col = c * 32 + 2 * e;
+          const float x = col < limit ? __uint_as_float(sv[2 * e]) : -CUDART_INF_F;
+          const float y = col + 1 < limit ? __uint_as_float(sv[2 * e + 1]) : -CUDART_INF_F;
+          const float a = ex2(fmaf(x, p.scale_log2, neg_m));
+          const float b = ex2(fmaf(y, p.scale_log2, neg_m));
+          l += a + b;
+          pk[e] = pack_bf16x2(a, b);
+        }
+        tmem_st16(t_s + c * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[g]);
+    }
+    if (ok) ok = wait_parity(&bars->o_full[g], 0, abort, p.timeout_ns);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = q_row < hd.lq;
+      const int64_t grow = row_base + q_row;
+      const float inv = 1.f / l;
+      __nv_bfloat16* op = p.out + (grow * p.h_q + me.head) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        if (valid) {
+          int4* dst = reinterpret_cast<int4*>(op + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_int4(int(pk[4 * v]), int(pk[4 * v + 1]), int(pk[4 * v + 2]), int(pk[4 * v + 3]));
+        }
+      }
+      if (valid && p.lse) p.lse[grow * p.h_q + me.head] = (m + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && bars->abort && p.status) {
+    atomicOr(p.status, 1);
+    __threadfence();
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+zz_status_t get_encoder() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q{};
+    void* fn = nullptr;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode)
+    return fail(ZZ_ERR_CUDA, std::string("cuTensorMapEncodeTiled unavailable: ") + cudaGetErrorString(err));
+  return ZZ_OK;
+}
+
+// 3-D bf16 tensor [rows][heads][d] seen as (d, heads, rows); box (64, 1, box_rows), 128B swizzle.
+zz_status_t encode_3d(CUtensorMap* m, const void* base, int d, int heads, int64_t rows, int box_rows) {
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(heads), cuuint64_t(rows)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(d) * heads * 2};
+  cuuint32_t box[3] = {64, 1, cuuint32_t(box_rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ZZ_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
+  return ZZ_OK;
+}
+
+template <int D>
+zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, const void* q,
+                        const void* k_pool, const void* v_pool, int64_t num_slots,
+                        const int32_t* page_table, int max_pages, int page_size, void* out,
+                        float* lse, int h_q, int h_kv, float scale, cudaStream_t stream) {
+  using C = Cfg<D>;
+  if (zz_status_t e = get_encoder()) return e;
+  const int box_rows = page_size >= 128 ? 128 : page_size;
+  CUtensorMap tq, tk, tv;
+  const int64_t q_rows = int64_t(rank_count) * pl->M;
+  if (zz_status_t e = encode_3d(&tq, q, D, h_q, q_rows, 128)) return e;
+  if (zz_status_t e = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return e;
+  if (zz_status_t e = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return e;
+  const char* ws = static_cast<const char*>(pl->dev_ws);
+  Params p{};
+  p.halves = reinterpret_cast<const HalfDesc*>(ws + pl->ws.halves);
+  p.page_table = page_table;
+  p.k_pool = static_cast<const __nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<const __nv_bfloat16*>(v_pool);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.status = reinterpret_cast<int*>(const_cast<char*>(ws) + pl->ws.status);
+  p.num_slots = num_slots;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.group = h_q / h_kv;
+  p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
+  p.head_groups = p.pair_heads ? h_q / 2 : h_q;
+  p.M = pl->M;
+  p.rank_begin = rank_begin;
+  p.max_pages = max_pages;
+  p.page_size = page_size;
+  p.box_rows = box_rows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = 1000000000ull;   // 1 s per wait
+  int64_t n_items;
+  const bool all = rank_count == pl->c;
+  if (p.pair_heads) {
+    p.items = reinterpret_cast<const WorkItem*>(ws + (all ? pl->ws.tiles_all : pl->ws.tiles_rank)) +
+              (all ? 0 : pl->tile_rank_off[rank_begin]);
+    n_items = all ? int64_t(pl->tiles_all.size())
+                  : pl->tile_rank_off[rank_begin + rank_count] - pl->tile_rank_off[rank_begin];
+  } else {
+    p.items = reinterpret_cast<const WorkItem*>(ws + (all ? pl->ws.pairs_all : pl->ws.pairs_rank)) +
+              (all ? 0 : pl->pair_rank_off[rank_begin]);
+    n_items = all ? int64_t(pl->pairs_all.size())
+                  : pl->pair_rank_off[rank_begin + rank_count] - pl->pair_rank_off[rank_begin];
+  }
+  const int64_t grid = n_items * p.head_groups;
+  if (grid == 0) return ZZ_OK;
+  if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: grid too large");
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    attr_set = true;
+  }
+  attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));
+  return ZZ_OK;
+}
+
+bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
+
+}  // namespace
+}  // namespace zz
+
+extern "C" zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_count,
+                                       const void* q, const void* k_pool, const void* v_pool,
+                                       int64_t num_slots, const int32_t* page_table, int max_pages,
+                                       int page_size, void* out, float* lse, int h_q, int h_kv, int d,
+                                       float softmax_scale, zz_dtype_t dtype, void* stream) {
+  using namespace zz;
+  if (!plan || !q || !k_pool || !v_pool || !page_table || !out)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: NULL argument");
+  if (h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: num_heads (" + std::to_string(h_q) +
+                                        ") must be a multiple of num_kv_heads (" + std::to_string(h_kv) + ")");
+  if (!plan->dev_ws) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: plan not uploaded");
+  if (rank_count <= 0 || rank_begin < 0 || rank_begin + rank_count > plan->c)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: rank range outside [0, cp_size)");
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: pointers must be 16-byte aligned");
+  if (page_size <= 0 || max_pages <= 0 || num_slots <= 0)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: page_size, max_pages and num_slots must be positive");
+  for (int s = 0; s < plan->bs; ++s) {
+    int32_t kv_max = 0;
+    for (int r = 0; r < plan->c; ++r) kv_max = std::max(kv_max, plan->kv_next[r][s]);
+    if ((int64_t(kv_max) + page_size - 1) / page_size > max_pages)
+      return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: page_table rows shorter than the kv lengths need");
+  }
+  if (d != 64 && d != 128) return fail(ZZ_ERR_UNSUPPORTED, "zz_attn_prefill: head_dim must be 64 or 128");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
+  auto s = static_cast<cudaStream_t>(stream);
+  if (dtype == ZZ_FP32)
+    return launch_attn_simt_fp32(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
+                                 max_pages, page_size, out, lse, h_q, h_kv, d, scale, s);
+  if (dtype != ZZ_BF16) return fail(ZZ_ERR_UNSUPPORTED, "zz_attn_prefill: dtype must be bf16 or fp32");
+  const bool ps_ok = page_size == 8 || page_size == 16 || page_size == 32 || page_size == 64 ||
+                     page_size % 128 == 0;
+  if (!ps_ok)
+    return fail(ZZ_ERR_UNSUPPORTED, "zz_attn_prefill: bf16 page_size must be 8, 16, 32, 64 or a multiple of 128");
+  if (d == 128)
+    return launch_bf16<128>(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
+                            max_pages, page_size, out, lse, h_q, h_kv, scale, s);
+  return launch_bf16<64>(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
+                         max_pages, page_size, out, lse, h_q, h_kv, scale, s);
+}

@@ -12,11 +12,15 @@
 //     (identical causal extent), or
 //   * otherwise: two consecutive row tiles of one head (the second one sees
 //     one more K/V tile at most).
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for sub-tile 0   (thread = TMEM lane = query row)
 //   warps 4-7  softmax for sub-tile 1
 //   warp  8    MMA issue (one thread) + TMEM allocation
 //   warp  9    TMA producer: Q once, then K_j, V_j into a ring of smem slots
+//   warps 10-11 idle
+// Launched at 168 registers a thread; the softmax warpgroups grow to 208 and
+// the third warpgroup shrinks to 88 (208 + 208 + 88 = 3 x 168 per SM
+// sub-partition), so a whole 128-column row of S stays in registers.
 // TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [256+D,256+2D).
 // P (bf16, two per column) overwrites the first 64 columns of its S tile and
 // feeds the P.V MMA straight from TMEM.  The MMA order per K/V tile j is
@@ -49,7 +53,8 @@ namespace {
 
 using namespace zz::dev;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
 constexpr int kWarpMma = 8;
 constexpr int kWarpLoad = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -174,6 +179,9 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  if (warp >= 8) {
+  // Third warpgroup: one setmaxnreg for all four warps, then per-warp roles.
+  regs_dec<kRegsOther>();
   if (warp == kWarpLoad) {
     // ================= TMA producer =================
     const int32_t* pt = p.page_table + int64_t(hd.seq) * p.max_pages;
@@ -329,8 +337,10 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       drain_parity(&bars->mma_done, 0, p.timeout_ns);
     }
     __syncwarp();
+  }   // warps 10-11 have no role
   } else {
     // ================= softmax + epilogue (warps 0-7) =================
+    regs_inc<kRegsSoftmax>();
     const int g = warp >> 2;                   // sub-tile
     const SubTile& me = st[g];
     const int quarter = warp & 3;
@@ -340,27 +350,29 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t t_o = tmem + lane_off + (g ? C::kColO1 : C::kColO0);
     const int q_row = me.q0 + r;
     const int my_pos = hd.kv_pos0 + q_row;     // last visible key (inclusive)
+    const int first_pos = hd.kv_pos0 + me.q0;  // position of the sub-tile's first row
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = me.n > 0;
     for (int j = 0; j < me.n && ok; ++j) {
       if (!(ok = wait_parity(&bars->s_full[g], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
       tc_fence_after();
-      // Pass 1: row maximum over the visible columns (S read 64 columns at a time).
-      const int limit = my_pos - j * 128 + 1;   // visible keys of this tile
-      float mx = -CUDART_INF_F;
+      // The whole 128-column row of S in registers: four loads, one wait.
+      uint32_t sr[128];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t a[32], b[32];
-        tmem_ld32(t_s + h * 64, a);
-        tmem_ld32(t_s + h * 64 + 32, b);
-        tmem_wait_ld();
+      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_wait_ld();
+      // Causal mask, only on tiles that reach past the sub-tile's first row.
+      if (j * 128 + 127 > first_pos) {
+        const int limit = my_pos - j * 128 + 1;   // visible keys of this row in this tile
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float x = (h * 64 + e < limit) ? __uint_as_float(a[e]) : -CUDART_INF_F;
-          const float y = (h * 64 + 32 + e < limit) ? __uint_as_float(b[e]) : -CUDART_INF_F;
-          mx = fmaxf(mx, fmaxf(x, y));
-        }
+        for (int c = 0; c < 128; ++c)
+          if (c >= limit) sr[c] = 0xFF800000u;     // -inf
       }
+      float mx = fmax3(__uint_as_float(sr[0]), __uint_as_float(sr[1]), __uint_as_float(sr[2]));
+#pragma unroll
+      for (int c = 3; c < 127; c += 2)
+        mx = fmax3(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+      mx = fmaxf(mx, __uint_as_float(sr[127]));
       const float m_tile = mx * p.scale_log2;
       if (j == 0) {
         m = m_tile;
@@ -379,27 +391,26 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         m = m_tile;
       }
-      // Pass 2: P = 2^(s*scale*log2e - m), summed in fp32, packed to bf16 over
-      // the first 64 columns of S.  Columns are re-read before being overwritten.
-      const float neg_m = -m;
+      // P = 2^(s*scale*log2e - m): packed FMA, ex2, packed running sum, bf16
+      // pairs written over the first 64 columns of S.
+      const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nm2 = make_float2(-m, -m);
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(t_s + c * 32, sv);
-        tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int col = c * 32 + 2 * e;
-          const float x = col < limit ? __uint_as_float(sv[2 * e]) : -CUDART_INF_F;
-          const float y = col + 1 < limit ? __uint_as_float(sv[2 * e + 1]) : -CUDART_INF_F;
-          const float a = ex2(fmaf(x, p.scale_log2, neg_m));
-          const float b = ex2(fmaf(y, p.scale_log2, neg_m));
-          l += a + b;
-          pk[e] = pack_bf16x2(a, b);
+          float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2, nm2);
+          x.x = ex2(x.x);
+          x.y = ex2(x.y);
+          acc = fadd2(acc, x);
+          pk[e] = pack_bf16x2(x.x, x.y);
         }
         tmem_st16(t_s + c * 16, pk);
       }
+      l += acc.x + acc.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[g]);

@@ -182,6 +182,34 @@ zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_coun
                             int page_size, void* out, float* lse, int h_q, int h_kv, int d,
                             float softmax_scale, zz_dtype_t dtype, void* stream);
 
+/*
+ * zz_attn_prefill without a workspace (bf16 only).  The zigzag pages have no
+ * counterpart to this call; it exists for callers that cannot hand the library
+ * device memory they allocated themselves: code that must not call
+ * cudaMalloc (for example while a CUDA graph is being captured, or inside a
+ * runtime whose memory is owned by its own arena allocator), and callers that
+ * want no device allocation tied to the life of a plan.
+ *
+ * Same arguments and results as zz_attn_prefill.  zz_plan_upload is not
+ * needed: the half table, the work list and the status word are copied on
+ * `stream` into a file-scope __device__ array of 1 MiB that lives inside the
+ * library (every GPU that loads libzz keeps it until the process exits).  The
+ * call itself allocates nothing and calls no cudaMalloc or cudaFree.
+ *   - Plans whose tables need more than 1 MiB (half table plus work list,
+ *     about 130 000 work items) are rejected with ZZ_ERR_INVALID_ARG before
+ *     anything is enqueued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the one array and the last call's tables stay in it; the
+ *     status word is cleared by every call.  Calls whose work overlaps on the
+ *     GPU (other streams, other host threads) race on the array: serialise them.
+ */
+zz_status_t zz_attn_prefill_noalloc(const zz_plan_t* plan, int rank_begin, int rank_count,
+                                    const void* q, const void* k_pool, const void* v_pool,
+                                    int64_t num_slots, const int32_t* page_table, int max_pages,
+                                    int page_size, void* out, float* lse, int h_q, int h_kv, int d,
+                                    float softmax_scale, zz_dtype_t dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

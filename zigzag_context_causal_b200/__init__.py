@@ -79,6 +79,7 @@ _sig = {
                                        _P, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int, _P]),
 }
+_sig["zz_attn_prefill_noalloc"] = _sig["zz_attn_prefill"]
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res

@@ -550,6 +550,108 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
 
 bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
 
+// ---------------------------------------------------------------- allocation-free variant
+// Scratch of zz_attn_prefill_noalloc: the half table, the work list and the
+// status word live here instead of in a caller-allocated workspace.  Every GPU
+// that loads the library keeps this array until the process exits.
+constexpr size_t kStaticScratchBytes = size_t(1) << 20;   // 1 MiB
+__device__ __align__(256) static unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[256] = {};   // device address of g_static_scratch, per device ordinal
+
+// Device address of the static scratch on the current device.  The name of the
+// array is only a host-side stand-in; the address must come from the runtime.
+zz_status_t static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 256) return fail(ZZ_ERR_UNSUPPORTED, "device ordinal above 255");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(ZZ_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return ZZ_OK;
+}
+
+template <int D>
+zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_count, const void* q,
+                               const void* k_pool, const void* v_pool, int64_t num_slots,
+                               const int32_t* page_table, int max_pages, int page_size, void* out,
+                               float* lse, int h_q, int h_kv, float scale, cudaStream_t stream) {
+  using C = Cfg<D>;
+  const int group = h_q / h_kv;
+  const bool pair_heads = group % 2 == 0;
+  const bool all = rank_count == pl->c;
+  const std::vector<WorkItem>& list = pair_heads ? (all ? pl->tiles_all : pl->tiles_rank)
+                                                 : (all ? pl->pairs_all : pl->pairs_rank);
+  const std::vector<int32_t>& off = pair_heads ? pl->tile_rank_off : pl->pair_rank_off;
+  const size_t first = all ? 0 : size_t(off[rank_begin]);
+  const size_t n_items = all ? list.size() : size_t(off[rank_begin + rank_count] - off[rank_begin]);
+  // Layout inside the static array: [status | halves | work items].
+  const size_t halves_off = 256;
+  const size_t halves_bytes = pl->halves.size() * sizeof(HalfDesc);
+  const size_t items_off = (halves_off + halves_bytes + 255) & ~size_t(255);
+  const size_t need = items_off + n_items * sizeof(WorkItem);
+  if (need > kStaticScratchBytes)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: plan tables need " + std::to_string(need) +
+                                        " bytes, more than the static scratch of " +
+                                        std::to_string(kStaticScratchBytes) + " bytes");
+  if (n_items == 0) return ZZ_OK;
+  if (zz_status_t e = get_encoder()) return e;
+  void* base = nullptr;
+  if (zz_status_t e = static_scratch_address(&base)) return e;
+  char* sc = static_cast<char*>(base);
+  cudaError_t e = cudaMemsetAsync(sc, 0, 16, stream);   // status word starts at zero
+  if (e == cudaSuccess && halves_bytes)
+    e = cudaMemcpyAsync(sc + halves_off, pl->halves.data(), halves_bytes, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(sc + items_off, list.data() + first, n_items * sizeof(WorkItem),
+                        cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess)
+    return fail(ZZ_ERR_CUDA, std::string("zz_attn_prefill_noalloc: ") + cudaGetErrorString(e));
+  const int box_rows = page_size >= 128 ? 128 : page_size;
+  CUtensorMap tq, tk, tv;
+  if (zz_status_t st = encode_3d(&tq, q, D, h_q, int64_t(rank_count) * pl->M, 128)) return st;
+  if (zz_status_t st = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return st;
+  if (zz_status_t st = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return st;
+  Params p{};
+  p.halves = reinterpret_cast<const HalfDesc*>(sc + halves_off);
+  p.items = reinterpret_cast<const WorkItem*>(sc + items_off);
+  p.status = reinterpret_cast<int*>(sc);
+  p.page_table = page_table;
+  p.k_pool = static_cast<const __nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<const __nv_bfloat16*>(v_pool);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.num_slots = num_slots;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.group = group;
+  p.pair_heads = pair_heads ? 1 : 0;
+  p.head_groups = pair_heads ? h_q / 2 : h_q;
+  p.M = pl->M;
+  p.rank_begin = rank_begin;
+  p.max_pages = max_pages;
+  p.page_size = page_size;
+  p.box_rows = box_rows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = 1000000000ull;
+  const int64_t grid = int64_t(n_items) * p.head_groups;
+  if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: grid too large");
+  e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+  attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));
+  return ZZ_OK;
+}
+
 }  // namespace
 }  // namespace zz
 
@@ -594,4 +696,47 @@ extern "C" zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, in
                             max_pages, page_size, out, lse, h_q, h_kv, scale, s);
   return launch_bf16<64>(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
                          max_pages, page_size, out, lse, h_q, h_kv, scale, s);
+}
+
+// Allocation-free variant of zz_attn_prefill (bf16): same arguments, but the
+// plan's device tables go into the library's static scratch array instead of
+// the workspace given to zz_plan_upload (which need not have been called).
+extern "C" zz_status_t zz_attn_prefill_noalloc(const zz_plan_t* plan, int rank_begin, int rank_count,
+                                               const void* q, const void* k_pool, const void* v_pool,
+                                               int64_t num_slots, const int32_t* page_table,
+                                               int max_pages, int page_size, void* out, float* lse,
+                                               int h_q, int h_kv, int d, float softmax_scale,
+                                               zz_dtype_t dtype, void* stream) {
+  using namespace zz;
+  if (!plan || !q || !k_pool || !v_pool || !page_table || !out)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: NULL argument");
+  if (h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: num_heads (" + std::to_string(h_q) +
+                                        ") must be a multiple of num_kv_heads (" + std::to_string(h_kv) + ")");
+  if (rank_count <= 0 || rank_begin < 0 || rank_begin + rank_count > plan->c)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: rank range outside [0, cp_size)");
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: pointers must be 16-byte aligned");
+  if (page_size <= 0 || max_pages <= 0 || num_slots <= 0)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: page_size, max_pages and num_slots must be positive");
+  for (int s = 0; s < plan->bs; ++s) {
+    int32_t kv_max = 0;
+    for (int r = 0; r < plan->c; ++r) kv_max = std::max(kv_max, plan->kv_next[r][s]);
+    if ((int64_t(kv_max) + page_size - 1) / page_size > max_pages)
+      return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: page_table rows shorter than the kv lengths need");
+  }
+  if (dtype != ZZ_BF16) return fail(ZZ_ERR_UNSUPPORTED, "zz_attn_prefill_noalloc: dtype must be bf16");
+  if (d != 64 && d != 128) return fail(ZZ_ERR_UNSUPPORTED, "zz_attn_prefill_noalloc: head_dim must be 64 or 128");
+  const bool ps_ok = page_size == 8 || page_size == 16 || page_size == 32 || page_size == 64 ||
+                     page_size % 128 == 0;
+  if (!ps_ok)
+    return fail(ZZ_ERR_UNSUPPORTED, "zz_attn_prefill_noalloc: page_size must be 8, 16, 32, 64 or a multiple of 128");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
+  auto s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return launch_bf16_static<128>(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
+                                   max_pages, page_size, out, lse, h_q, h_kv, scale, s);
+  return launch_bf16_static<64>(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
+                                max_pages, page_size, out, lse, h_q, h_kv, scale, s);
 }

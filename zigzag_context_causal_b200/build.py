@@ -1,6 +1,7 @@
 """Build libzz.so in-tree with nvcc for sm_100a (no JIT, no torch extension).
 
-Usage: python -m zigzag_context_causal_b200.build   (or build() from Python)
+Usage: python zigzag_context_causal_b200/build.py   (or build() from Python;
+the package itself cannot be imported before the library exists)
 """
 from __future__ import annotations
 

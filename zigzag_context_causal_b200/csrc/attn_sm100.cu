@@ -16,7 +16,7 @@
 //   warps 0-3  softmax for sub-tile 0   (thread = TMEM lane = query row)
 //   warps 4-7  softmax for sub-tile 1
 //   warp  8    MMA issue (one thread) + TMEM allocation
-//   warp  9    TMA producer: Q once, then K_j, V_j into a ring of smem slots
+//   warp  9    TMA producer: Q once, then K/V stages (V_{j-1}, K_j) into a smem ring
 //   warps 10-11 idle
 // Launched at 168 registers a thread; the softmax warpgroups grow to 208 and
 // the third warpgroup shrinks to 88 (208 + 208 + 88 = 3 x 168 per SM
@@ -39,6 +39,7 @@
 #include <string>
 
 #include "ptx_sm100.cuh"
+#include "exp2_poly.h"
 #include "zz_internal.h"
 
 namespace zz {
@@ -59,16 +60,24 @@ constexpr int kWarpMma = 8;
 constexpr int kWarpLoad = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 256 between rescales
+// Of the 16 exponential pairs of each 32-column chunk, pairs >= kPolyFrom are
+// evaluated with the FMA-pipe polynomial, the rest with MUFU ex2.  Measured on
+// B200 with this pipeline, sending 25% to the polynomial (kPolyFrom = 12) was
+// ~5% slower than MUFU alone, so all pairs use ex2 (kPolyFrom = 16).
+constexpr int kPolyFrom = 16;
 
 template <int D>
 struct Cfg {
   static constexpr int kBoxes = D / 64;                  // 128-byte swizzle boxes per row
   static constexpr int kBoxBytes = 128 * 128;            // 128 rows x 128 bytes
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one Q, K or V tile
-  static constexpr int kSlots = D == 64 ? 8 : 4;         // K/V ring depth
+  // K/V ring: stage t holds K_t (second half) and V_{t-1} (first half), the two
+  // tiles the MMA issuer consumes in the same iteration.
+  static constexpr int kStages = D == 64 ? 4 : 2;
+  static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kStageBytes;
   static constexpr int kSmem = kBarOff + 512 + 1024;     // + barriers + alignment slack
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
 };
@@ -86,6 +95,9 @@ struct Params {
   int h_q, h_kv, group;
   int pair_heads;       // 1: sub-tiles are heads 2g, 2g+1; 0: row tiles 2t, 2t+1 of head g
   int head_groups;      // CTAs per work item
+  int groups_per_kv;    // head groups that read the same K/V head
+  int chunk_items;      // work items per scheduling chunk (see block_coords)
+  int n_items;
   int M, rank_begin;
   int max_pages, page_size, box_rows;
   float scale_log2;
@@ -130,8 +142,22 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int lane = threadIdx.x & 31;
 
   // ---- work decomposition ----
-  const WorkItem w = p.items[blockIdx.x / p.head_groups];
-  const int hg = blockIdx.x % p.head_groups;
+  // Blocks run in index order.  Items are taken in chunks of chunk_items
+  // (longest first); inside a chunk the blocks go K/V head by K/V head, so a
+  // wave of resident CTAs is many items x the query heads of ONE K/V head, all
+  // streaming the same K/V tiles at about the same time (L2 reuse).
+  int item_idx, hg;
+  {
+    const int per_chunk = p.chunk_items * p.head_groups;
+    const int chunk = blockIdx.x / per_chunk;
+    const int r = blockIdx.x - chunk * per_chunk;
+    const int w_items = min(p.chunk_items, p.n_items - chunk * p.chunk_items);
+    const int kvh = r / (w_items * p.groups_per_kv);
+    const int r2 = r - kvh * w_items * p.groups_per_kv;
+    item_idx = chunk * p.chunk_items + r2 / p.groups_per_kv;
+    hg = kvh * p.groups_per_kv + r2 % p.groups_per_kv;
+  }
+  const WorkItem w = p.items[item_idx];
   const HalfDesc hd = p.halves[w.half_id];
   SubTile st[2];
   if (p.pair_heads) {
@@ -156,7 +182,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&bars->o_full[i], 1);
     }
     mbar_init(&bars->mma_done, 1);
-    for (int s = 0; s < C::kSlots; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
@@ -197,21 +223,24 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                       int32_t(row_base + st[i].q0));
       }
     }
-    int load_no = 0;
     const int chunks = 128 / p.box_rows;
-    for (int j = 0; j < n_max && !*abort; ++j) {
-      for (int t = 0; t < 2; ++t, ++load_no) {
-        const int slot = load_no % C::kSlots;
-        const uint32_t use = load_no / C::kSlots;
-        if (!wait_parity(&bars->kv_empty[slot], (use & 1u) ^ 1u, abort, p.timeout_ns)) break;
-        uint8_t* tile = smem + C::kKVOff + slot * C::kTileBytes;
-        const __nv_bfloat16* pool = t == 0 ? p.k_pool : p.v_pool;
-        const void* tm = t == 0 ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
-        const int key0 = j * 128;
+    // Stage t (t = 0 .. n_max): K_t if t < n_max, V_{t-1} if t >= 1.
+    int t = 0;
+    for (; t <= n_max && !*abort; ++t) {
+      const int slot = t % C::kStages;
+      const uint32_t use = t / C::kStages;
+      if (!wait_parity(&bars->kv_empty[slot], (use & 1u) ^ 1u, abort, p.timeout_ns)) break;
+      uint8_t* stage = smem + C::kKVOff + slot * C::kStageBytes;
+      uint32_t tma_bytes = 0;
+      for (int which = 0; which < 2; ++which) {       // 0: V_{t-1} (first half), 1: K_t (second half)
+        const int tile_j = which ? t : t - 1;
+        if (tile_j < 0 || tile_j >= n_max) continue;
+        uint8_t* tile = stage + which * C::kTileBytes;
+        const __nv_bfloat16* pool = which ? p.k_pool : p.v_pool;
+        const int key0 = tile_j * 128;
         // Rows at or beyond kv_len (end of the sequence's keys) are filled by
         // hand: real keys copied, the rest zero, so no stale or unwritten pool
         // slot can reach the MMAs (0 * NaN would poison P.V).
-        uint32_t tma_bytes = 0;
         bool manual = false;
         for (int c = 0; c < chunks; ++c) {
           if (key0 + (c + 1) * p.box_rows <= hd.kv_len) tma_bytes += p.box_rows * 128 * C::kBoxes;
@@ -239,8 +268,15 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           fence_proxy_async_smem();
           __syncwarp();
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&bars->kv_full[slot], tma_bytes);
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->kv_full[slot], tma_bytes);
+        for (int which = 0; which < 2; ++which) {
+          const int tile_j = which ? t : t - 1;
+          if (tile_j < 0 || tile_j >= n_max) continue;
+          uint8_t* tile = stage + which * C::kTileBytes;
+          const void* tm = which ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
+          const int key0 = tile_j * 128;
           for (int c = 0; c < chunks; ++c) {
             const int kc = key0 + c * p.box_rows;
             if (kc + p.box_rows > hd.kv_len) continue;
@@ -250,87 +286,78 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                           b * 64, kv_head, slot0);
           }
         }
-        __syncwarp();
       }
+      __syncwarp();
     }
+    const int load_no = t;   // stages issued
     // Never leave with copies in flight into shared memory.
     if (lane == 0) {
-      for (int n = max(0, load_no - C::kSlots); n < load_no; ++n)
-        drain_parity(&bars->kv_full[n % C::kSlots], (uint32_t(n / C::kSlots)) & 1u, p.timeout_ns);
+      for (int n = max(0, load_no - C::kStages); n < load_no; ++n)
+        drain_parity(&bars->kv_full[n % C::kStages], (uint32_t(n / C::kStages)) & 1u, p.timeout_ns);
       for (int i = 0; i < 2; ++i)
         if (q_issued[i]) drain_parity(&bars->q_full[i], 0, p.timeout_ns);
     }
   } else if (warp == kWarpMma) {
     // ================= MMA issue (single thread) =================
+    // A single thread retires a tcgen05.mma only every ~50 cycles, little faster
+    // than a 128x128x16 MMA executes (64 cycles), so everything else this thread
+    // does between MMAs (barrier waits, commits) must stay short: descriptors
+    // are a base plus a compile-time offset, the sub-tile code is unrolled, and
+    // each K/V tile costs one full-wait and one release (stage = V_j + K_{j+1}).
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_addr = smem_u32(smem + C::kQOff);
       const uint32_t kv_addr = smem_u32(smem + C::kKVOff);
-      const uint32_t col_s[2] = {C::kColS0, C::kColS1};
-      const uint32_t col_o[2] = {C::kColO0, C::kColO1};
-      auto slot_of = [](int n) { return n % C::kSlots; };
-      auto par_of = [](int n) { return uint32_t(n / C::kSlots) & 1u; };
-      auto issue_s = [&](int i, int slot) {
-        const uint32_t qa = q_addr + i * C::kTileBytes;
-        const uint32_t ka = kv_addr + slot * C::kTileBytes;
+      // K-major operands (Q, K): SBO = 8 rows x 128 B; MN-major V: LBO = next 64-column box.
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+      const uint64_t dq1 = dq0 + uint64_t(C::kTileBytes >> 4);
+      const uint64_t dk0 = smem_desc_sw128(kv_addr + C::kTileBytes, 16, 1024);   // K half of stage 0
+      const uint64_t dv0 = smem_desc_sw128(kv_addr, C::kBoxBytes, 1024);         // V half of stage 0
+      const int n0 = st[0].n, n1 = st[1].n;
+      auto issue_s = [&](uint32_t col, uint64_t dq, int slot) {
+        const uint64_t dk = dk0 + uint64_t((slot * C::kStageBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + col_s[i], smem_desc_sw128(qa + off, 16, 1024),
-                 smem_desc_sw128(ka + off, 16, 1024), idesc_s, kk > 0);
+          const uint64_t off = uint64_t(((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4);
+          mma_ss(tmem + col, dq + off, dk + off, idesc_s, kk > 0);
         }
       };
-      auto issue_pv = [&](int i, int slot, bool acc) {
-        const uint32_t va = kv_addr + slot * C::kTileBytes;
+      auto issue_pv = [&](uint32_t col_o, uint32_t col_p, int slot, bool acc) {
+        const uint64_t dv = dv0 + uint64_t((slot * C::kStageBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + col_o[i], tmem + col_s[i] + kk * 8,
-                 smem_desc_sw128(va + kk * 2048, C::kBoxBytes, 1024), idesc_o, acc || kk > 0);
+          mma_ts(tmem + col_o, tmem + col_p + kk * 8, dv + uint64_t((kk * 2048) >> 4), idesc_o,
+                 (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = true;
-      for (int i = 0; i < 2 && ok; ++i)
-        if (st[i].n) ok = wait_parity(&bars->q_full[i], 0, abort, p.timeout_ns);
-      if (ok && n_max > 0) ok = wait_parity(&bars->kv_full[slot_of(0)], par_of(0), abort, p.timeout_ns);
-      if (ok && n_max > 0) {
+      if (n0) ok = wait_parity(&bars->q_full[0], 0, abort, p.timeout_ns);
+      if (ok && n1) ok = wait_parity(&bars->q_full[1], 0, abort, p.timeout_ns);
+      if (ok) ok = wait_parity(&bars->kv_full[0], 0, abort, p.timeout_ns);   // stage 0: K_0
+      if (ok) {
         tc_fence_after();
-        for (int i = 0; i < 2; ++i)
-          if (st[i].n) {
-            issue_s(i, slot_of(0));
-            mma_commit(&bars->s_full[i]);
-          }
-        mma_commit(&bars->kv_empty[slot_of(0)]);
+        if (n0) { issue_s(C::kColS0, dq0, 0); mma_commit(&bars->s_full[0]); }
+        if (n1) { issue_s(C::kColS1, dq1, 0); mma_commit(&bars->s_full[1]); }
+        mma_commit(&bars->kv_empty[0]);
       }
       for (int j = 0; j < n_max && ok; ++j) {
-        const int nv = 2 * j + 1, nk = 2 * j + 2;
-        if (!(ok = wait_parity(&bars->kv_full[slot_of(nv)], par_of(nv), abort, p.timeout_ns))) break;
-        tc_fence_after();
-        bool k_ready = false;
-        for (int i = 0; i < 2 && ok; ++i) {
-          if (j >= st[i].n) continue;
-          if (!(ok = wait_parity(&bars->p_full[i], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+        const int t = j + 1;                    // stage with V_j and K_{j+1}
+        const int slot = t % C::kStages;
+        if (!(ok = wait_parity(&bars->kv_full[slot], uint32_t(t / C::kStages) & 1u, abort, p.timeout_ns))) break;
+        if (j < n0) {
+          if (!(ok = wait_parity(&bars->p_full[0], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
           tc_fence_after();
-          issue_pv(i, slot_of(nv), j > 0);
-          if (j == st[i].n - 1) mma_commit(&bars->o_full[i]);
-          if (j + 1 < st[i].n) {
-            if (!k_ready) {
-              if (!(ok = wait_parity(&bars->kv_full[slot_of(nk)], par_of(nk), abort, p.timeout_ns))) break;
-              tc_fence_after();
-              k_ready = true;
-            }
-            issue_s(i, slot_of(nk));
-            mma_commit(&bars->s_full[i]);
-          }
+          issue_pv(C::kColO0, C::kColS0, slot, j > 0);
+          if (j == n0 - 1) mma_commit(&bars->o_full[0]);
+          else { issue_s(C::kColS0, dq0, slot); mma_commit(&bars->s_full[0]); }
         }
-        if (!ok) break;
-        mma_commit(&bars->kv_empty[slot_of(nv)]);
-        if (j + 1 < n_max) {
-          if (!k_ready) {  // the next K tile is only used by the longer sub-tile
-            if (!(ok = wait_parity(&bars->kv_full[slot_of(nk)], par_of(nk), abort, p.timeout_ns))) break;
-            tc_fence_after();
-          }
-          mma_commit(&bars->kv_empty[slot_of(nk)]);
+        if (j < n1) {
+          if (!(ok = wait_parity(&bars->p_full[1], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+          tc_fence_after();
+          issue_pv(C::kColO1, C::kColS1, slot, j > 0);
+          if (j == n1 - 1) mma_commit(&bars->o_full[1]);
+          else { issue_s(C::kColS1, dq1, slot); mma_commit(&bars->s_full[1]); }
         }
+        mma_commit(&bars->kv_empty[slot]);
       }
       // Drain: no MMA may still be running when TMEM is released.
       mma_commit(&bars->mma_done);
@@ -368,11 +395,17 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int c = 0; c < 128; ++c)
           if (c >= limit) sr[c] = 0xFF800000u;     // -inf
       }
-      float mx = fmax3(__uint_as_float(sr[0]), __uint_as_float(sr[1]), __uint_as_float(sr[2]));
+      // Row maximum as 8 independent max3 chains (short dependency depth).
+      float pm[8];
 #pragma unroll
-      for (int c = 3; c < 127; c += 2)
-        mx = fmax3(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-      mx = fmaxf(mx, __uint_as_float(sr[127]));
+      for (int q = 0; q < 8; ++q) pm[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
+#pragma unroll
+      for (int c = 16; c < 128; c += 16)
+#pragma unroll
+        for (int q = 0; q < 8; q += 2)
+          pm[q] = fmax3(pm[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + q + 8])),
+          pm[q + 1] = fmax3(pm[q + 1], __uint_as_float(sr[c + q + 1]), __uint_as_float(sr[c + q + 9]));
+      const float mx = fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], fmax3(pm[5], pm[6], pm[7])));
       const float m_tile = mx * p.scale_log2;
       if (j == 0) {
         m = m_tile;
@@ -395,7 +428,8 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // pairs written over the first 64 columns of S.
       const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
       const float2 nm2 = make_float2(-m, -m);
-      float2 acc = make_float2(0.f, 0.f);
+      float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -403,13 +437,18 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int e = 0; e < 16; ++e) {
           const int col = c * 32 + 2 * e;
           float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2, nm2);
-          x.x = ex2(x.x);
-          x.y = ex2(x.y);
-          acc = fadd2(acc, x);
+          if (e >= kPolyFrom) {
+            x = exp2_poly2(x);
+          } else {
+            x.x = ex2(x.x);
+            x.y = ex2(x.y);
+          }
+          acc4[e & 3] = fadd2(acc4[e & 3], x);
           pk[e] = pack_bf16x2(x.x, x.y);
         }
         tmem_st16(t_s + c * 16, pk);
       }
+      const float2 acc = fadd2(fadd2(acc4[0], acc4[1]), fadd2(acc4[2], acc4[3]));
       l += acc.x + acc.y;
       tmem_wait_st();
       tc_fence_before();
@@ -485,6 +524,18 @@ zz_status_t encode_3d(CUtensorMap* m, const void* base, int d, int heads, int64_
   return ZZ_OK;
 }
 
+// Items per scheduling chunk: enough that one K/V head's blocks of a chunk
+// fill every SM once (one resident CTA per SM).
+int chunk_items_for(int groups_per_kv) {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+  }
+  return std::max(1, (sms + groups_per_kv - 1) / groups_per_kv);
+}
+
 template <int D>
 zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, const void* q,
                         const void* k_pool, const void* v_pool, int64_t num_slots,
@@ -513,6 +564,7 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
   p.group = h_q / h_kv;
   p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
   p.head_groups = p.pair_heads ? h_q / 2 : h_q;
+  p.groups_per_kv = p.pair_heads ? p.group / 2 : p.group;
   p.M = pl->M;
   p.rank_begin = rank_begin;
   p.max_pages = max_pages;
@@ -536,6 +588,8 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
   const int64_t grid = n_items * p.head_groups;
   if (grid == 0) return ZZ_OK;
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: grid too large");
+  p.n_items = int(n_items);
+  p.chunk_items = chunk_items_for(p.groups_per_kv);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
@@ -549,6 +603,7 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
 }
 
 bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
+
 
 // ---------------------------------------------------------------- allocation-free variant
 // Scratch of zz_attn_prefill_noalloc: the half table, the work list and the
@@ -635,6 +690,7 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   p.group = group;
   p.pair_heads = pair_heads ? 1 : 0;
   p.head_groups = pair_heads ? h_q / 2 : h_q;
+  p.groups_per_kv = pair_heads ? group / 2 : group;
   p.M = pl->M;
   p.rank_begin = rank_begin;
   p.max_pages = max_pages;
@@ -644,6 +700,8 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   p.timeout_ns = 1000000000ull;
   const int64_t grid = int64_t(n_items) * p.head_groups;
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: grid too large");
+  p.n_items = int(n_items);
+  p.chunk_items = chunk_items_for(p.groups_per_kv);
   e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
   attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);

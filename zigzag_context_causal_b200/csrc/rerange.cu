@@ -34,61 +34,68 @@ __device__ __forceinline__ void st_stream(int4* p, int4 v) {
                : "memory");
 }
 
-// One launch moves `ntensors` (1 or 2) tensors of `rows` rows each.  Vector v
-// of the flattened [tensor][row][vec] space: dst row = dst_map(row), src row =
-// src_map(row).  `vec_shift` = log2(vectors per row) when that is a power of
-// two, else -1.
+// One launch moves `ntensors` (1 or 2) tensors of `rows` rows each.  Vector e
+// of the flattened [tensor][row][vec] space goes from row src_map(row) of the
+// source to row dst_map(row) of the destination.  The maps are compile-time
+// choices (identity, int32 table, int64 table) so that the per-vector work is
+// a shift, a mask, two cached index loads and the 16-byte copy.
 struct MoveArgs {
   const int4* src[2];
   int4* dst[2];
-  const int32_t* src_idx;  // nullptr = identity
-  const int32_t* dst_idx32;  // one of dst_idx32 / dst_idx64 / neither (identity)
+  const int32_t* src_idx;    // natural token -> source row (nullptr: identity)
+  const int32_t* dst_idx32;  // destination row tables (one of them, or identity)
   const int64_t* dst_idx64;
   int64_t rows;
   int64_t vecs_per_row;
-  int vec_shift;
+  int vec_shift;             // log2(vecs_per_row), or -1 when not a power of two
   int ntensors;
-  int64_t dst_rows;  // rows of the destination, out-of-range rows are skipped
+  int64_t dst_rows;          // rows of the destination; out-of-range rows are skipped
 };
 
+enum DstKind { kDstIdentity = 0, kDstI32 = 1, kDstI64 = 2 };
+
+template <bool kSrcTable, int kDst, bool kPow2>
 __global__ void __launch_bounds__(kThreads) move_rows_kernel(MoveArgs a) {
   const int64_t per_tensor = a.rows * a.vecs_per_row;
   const int64_t total = per_tensor * a.ntensors;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; i < total; i += stride * kUnroll) {
+  const int64_t vmask = a.vecs_per_row - 1;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride * kUnroll) {
     int4 val[kUnroll];
     int4* dptr[kUnroll];
+    // The 16-byte load depends only on the source index (rows of the plan,
+    // valid by construction); the destination index is checked only to
+    // predicate the store, so loads never wait on it.
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t e = i + u * stride;
       dptr[u] = nullptr;
       if (e < total) {
-        const int tsel = e >= per_tensor;
-        const int64_t f = e - (tsel ? per_tensor : 0);
-        int64_t row, vec;
-        if (a.vec_shift >= 0) {
-          row = f >> a.vec_shift;
-          vec = f & (a.vecs_per_row - 1);
-        } else {
-          row = f / a.vecs_per_row;
-          vec = f - row * a.vecs_per_row;
-        }
-        const int64_t srow = a.src_idx ? int64_t(__ldg(a.src_idx + row)) : row;
-        const int64_t drow = a.dst_idx64 ? __ldg(a.dst_idx64 + row)
-                             : a.dst_idx32 ? int64_t(__ldg(a.dst_idx32 + row)) : row;
-        if (drow >= 0 && drow < a.dst_rows) {
-          const int4* sb = tsel ? a.src[1] : a.src[0];
-          int4* db = tsel ? a.dst[1] : a.dst[0];
-          val[u] = ld_stream(sb + srow * a.vecs_per_row + vec);
-          dptr[u] = db + drow * a.vecs_per_row + vec;
-        }
+        const bool second = e >= per_tensor;
+        const int64_t f = second ? e - per_tensor : e;
+        const int64_t row = kPow2 ? (f >> a.vec_shift) : f / a.vecs_per_row;
+        const int64_t vec = kPow2 ? (f & vmask) : f - row * a.vecs_per_row;
+        const int64_t srow = kSrcTable ? int64_t(__ldg(a.src_idx + row)) : row;
+        const int64_t drow = kDst == kDstI64 ? __ldg(a.dst_idx64 + row)
+                             : kDst == kDstI32 ? int64_t(__ldg(a.dst_idx32 + row)) : row;
+        const int4* sb = second ? a.src[1] : a.src[0];
+        int4* db = second ? a.dst[1] : a.dst[0];
+        const int64_t soff = kPow2 ? (srow << a.vec_shift) : srow * a.vecs_per_row;
+        const int64_t doff = kPow2 ? (drow << a.vec_shift) : drow * a.vecs_per_row;
+        val[u] = ld_stream(sb + soff + vec);
+        if (kDst == kDstIdentity || (drow >= 0 && drow < a.dst_rows)) dptr[u] = db + doff + vec;
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u)
       if (dptr[u]) st_stream(dptr[u], val[u]);
   }
+}
+
+template <bool kSrcTable, int kDst>
+void launch_kind(const MoveArgs& a, unsigned blocks, cudaStream_t s) {
+  if (a.vec_shift >= 0) move_rows_kernel<kSrcTable, kDst, true><<<blocks, kThreads, 0, s>>>(a);
+  else move_rows_kernel<kSrcTable, kDst, false><<<blocks, kThreads, 0, s>>>(a);
 }
 
 zz_status_t launch_move(const MoveArgs& a, cudaStream_t s) {
@@ -101,7 +108,10 @@ zz_status_t launch_move(const MoveArgs& a, cudaStream_t s) {
   int64_t blocks = int64_t(sms) * 8;
   const int64_t need = (total + int64_t(kThreads) * kUnroll - 1) / (int64_t(kThreads) * kUnroll);
   if (need < blocks) blocks = need;
-  move_rows_kernel<<<unsigned(blocks), kThreads, 0, s>>>(a);
+  const unsigned b = unsigned(blocks);
+  if (a.src_idx && a.dst_idx64) launch_kind<true, kDstI64>(a, b, s);        // rerange into the pool
+  else if (!a.src_idx && a.dst_idx32) launch_kind<false, kDstI32>(a, b, s);  // shard
+  else return zz::fail(ZZ_ERR_INVALID_ARG, "move_rows: unsupported index maps");
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return zz::fail(ZZ_ERR_CUDA, std::string("move_rows launch: ") + cudaGetErrorString(e));
   return ZZ_OK;

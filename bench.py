@@ -55,6 +55,24 @@ def _lens(spec):
     return list(spec)
 
 
+def rank_range(cp: int, world: int, rank: int):
+    """Virtual ranks [r0, r0 + r_per) owned by this process when c ranks are
+    spread over `world` GPUs (c must be a multiple of world)."""
+    if cp % world:
+        raise ValueError(f"cp_size {cp} must be a multiple of the GPU count {world}")
+    r_per = cp // world
+    return rank * r_per, r_per
+
+
+def all_gather_rows(dist, out, local):
+    """All-gather this process's rank-ordered rows into `out` ([c*M, ...]):
+    the exchange step of zigzag CP (K and V shards, in rank order)."""
+    if dist.get_backend() == "nccl":
+        dist.all_gather_into_tensor(out, local)
+    else:  # gloo (CPU tests): gather into views of `out`
+        dist.all_gather(list(out.chunk(dist.get_world_size())), local)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -224,10 +242,7 @@ def main_gpu(args):
 
     cp, spec, h_q, h_kv, d, ps, desc = WORKLOADS[args.workload]
     lens = _lens(spec)
-    if cp % world:
-        raise SystemExit(f"cp_size {cp} must be a multiple of the GPU count {world}")
-    r_per = cp // world
-    r0 = rank * r_per
+    r0, r_per = rank_range(cp, world, rank)
     T = sum(lens)
     plan = zz.Plan(cp, extend_lens=lens)
     M = plan.M
@@ -264,8 +279,8 @@ def main_gpu(args):
         # S1 plan tables, S3 (multi-GPU only) all-gather, S4 rerange, S5 attention
         plan.upload(ws)
         if world > 1:
-            dist.all_gather_into_tensor(k_g, k_local)
-            dist.all_gather_into_tensor(v_g, v_local)
+            all_gather_rows(dist, k_g, k_local)
+            all_gather_rows(dist, v_g, v_local)
         e0, e1, e2 = ev(), ev(), ev()
         e0.record(stream)
         zz.rerange_kv_to_pool(plan, k_g, v_g, k_pool, v_pool, loc)
@@ -326,8 +341,8 @@ def main_gpu(args):
             k_d.copy_(k_h, non_blocking=True)
             v_d.copy_(v_h, non_blocking=True)
             if world > 1:
-                dist.all_gather_into_tensor(k_g, k_d)
-                dist.all_gather_into_tensor(v_g, v_d)
+                all_gather_rows(dist, k_g, k_d)
+                all_gather_rows(dist, v_g, v_d)
             plan.upload(ws)
             zz.rerange_kv_to_pool(plan, k_g, v_g, k_pool, v_pool, loc)
             zz.attn_prefill(plan, q_d, k_pool, v_pool, page_table, ps, out, softmax_scale=scale,

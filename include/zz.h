@@ -183,6 +183,17 @@ zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_coun
                             float softmax_scale, zz_dtype_t dtype, void* stream);
 
 /*
+ * Diagnostic: launch one thread that waits, with the same bounded mbarrier
+ * wait every pipeline stage of zz_attn_prefill uses, on a barrier that nothing
+ * arrives at.  The wait must give up after `timeout_ns` and the kernel must
+ * return normally, leaving the context usable.  Writes dev_status[0] = 1 when
+ * the wait gave up (0 if it returned early, which would be a bug) and
+ * dev_status[1] = elapsed nanoseconds.  dev_status: 2 x int64 device memory.
+ * ZZ_ERR_INVALID_ARG unless 0 < timeout_ns <= 10 s.
+ */
+zz_status_t zz_debug_wait_timeout(int64_t timeout_ns, int64_t* dev_status, void* stream);
+
+/*
  * zz_attn_prefill without a workspace (bf16 only).  The zigzag pages have no
  * counterpart to this call; it exists for callers that cannot hand the library
  * device memory they allocated themselves: code that must not call

@@ -1,0 +1,58 @@
+"""Edge cases and the error contract on the GPU."""
+import numpy as np
+import pytest
+import torch
+
+from tests.gpu_cases import Case, Run, assert_close, zz
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_full(run):
+    run.attend()
+    p = run.ref_plan
+    out = run.out.float().cpu().numpy()
+    for r in range(p.cp_size):
+        o_ref, _ = run.expected_rank(r)
+        n = p.per_rank_actual_token[r]
+        assert np.isfinite(out[r * p.M: r * p.M + n]).all()
+        assert_close(out[r * p.M: r * p.M + n], o_ref, run.case.dtype, f"rank {r}")
+    assert run.plan.device_status() == 0
+
+
+@pytest.mark.parametrize("case", [
+    Case(2, [4], 2, 1, 128, page_size=16),                     # every block is one token
+    Case(4, [8, 9, 15, 16, 17], 4, 2, 128, page_size=8),       # minimal and near-minimal lengths
+    Case(2, [5] * 40, 2, 2, 64, page_size=16),                 # many short sequences
+    Case(8, [257, 1000, 129], 6, 3, 128, page_size=32),        # odd group 3, c=8
+    Case(3, [129, 130], 2, 2, 128, page_size=128),             # tiles that end one row past a tile
+], ids=["blocks-of-one", "minimal", "bs40", "c8-g3", "ps128-ragged"])
+def test_edge_case_parity(case):
+    _check_full(Run(case))
+
+
+def test_unsupported_shapes_are_refused():
+    run = Run(Case(2, [64], 2, 2, 128, page_size=16))
+    with pytest.raises(zz.ZZError) as e:
+        zz.attn_prefill(run.plan, run.q_ranked, run.k_pool, run.v_pool, run.page_table, 24, run.out)
+    assert e.value.status == zz.ZZ_ERR_UNSUPPORTED
+    q96 = torch.zeros(run.q_ranked.shape[0], 2, 96, dtype=torch.bfloat16, device="cuda")
+    kv96 = torch.zeros(run.k_pool.shape[0], 2, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(zz.ZZError) as e:
+        zz.attn_prefill(run.plan, q96, kv96, kv96, run.page_table, 16, q96)
+    assert e.value.status == zz.ZZ_ERR_UNSUPPORTED
+    with pytest.raises(zz.ZZError) as e:        # page table too short for the kv lengths
+        zz.attn_prefill(run.plan, run.q_ranked, run.k_pool, run.v_pool, run.page_table[:, :1], 16,
+                        run.out)
+    assert e.value.status == zz.ZZ_ERR_INVALID_ARG
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable():
+    status = torch.zeros(2, dtype=torch.int64, device="cuda")
+    zz.debug_wait_timeout(50_000_000, status)               # 50 ms on a barrier nobody arrives at
+    torch.cuda.synchronize()
+    flag, ns = status.tolist()
+    assert flag == 1
+    assert 40_000_000 <= ns < 2_000_000_000
+    # the context still runs real work afterwards
+    _check_full(Run(Case(2, [200], 4, 2, 128, page_size=16)))

@@ -80,6 +80,7 @@ _sig = {
                                        ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int, _P]),
 }
 _sig["zz_attn_prefill_noalloc"] = _sig["zz_attn_prefill"]
+_sig["zz_debug_wait_timeout"] = (ctypes.c_int, [ctypes.c_int64, _P, _P])
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
@@ -232,3 +233,8 @@ def raw_call(name: str, *args) -> int:
 
 def last_error() -> str:
     return _lib.zz_last_error().decode()
+
+
+def debug_wait_timeout(timeout_ns: int, status: torch.Tensor, stream=None) -> None:
+    """Run the bounded-wait self test; ``status`` is an int64 CUDA tensor of 2."""
+    _check(_lib.zz_debug_wait_timeout(int(timeout_ns), _ptr(status), _stream(stream)))

@@ -128,12 +128,37 @@ zz_status_t zz_plan_device_status(const zz_plan_t* plan, int32_t* flags, int cle
 
 /*
  * Shard rows from natural token order into the rank-ordered padded layout
- * [c*M, row_bytes] (zigzag.py, shard_hidden_states for every rank, stacked as
- * _all_gather_reorganized would deliver them).  Padding rows are not written.
- * src: [T, row_bytes], dst: [c*M, row_bytes]; row_bytes a multiple of 16.
+ * [c*M, row_bytes] (zigzag.py, shard_hidden_states / shard_position_ids for
+ * every rank, stacked as _all_gather_reorganized would deliver them).
+ * Padding rows are not written.  src: [T, row_bytes], dst: [c*M, row_bytes].
+ * row_bytes: a multiple of 4 (16-byte rows and pointers take the wide path);
+ * pointers 4-byte aligned.  Position ids of shape [3, T] (mrope) are sharded
+ * as rows of their transpose [T, 3].
  */
 zz_status_t zz_shard_rows(const zz_plan_t* plan, const void* src, void* dst,
                           int64_t row_bytes, void* stream);
+
+/*
+ * Inverse of zz_shard_rows: dst[t] = src[row of token t], rank-ordered padded
+ * [c*M, row_bytes] back to token order [T, row_bytes] (zigzag.py,
+ * gather_hidden_states after the all-gather: trim, reverse split, cat).
+ * Same row/alignment rules as zz_shard_rows.
+ */
+zz_status_t zz_gather_rows(const zz_plan_t* plan, const void* src, void* dst,
+                           int64_t row_bytes, void* stream);
+
+/*
+ * One rank's zigzag shard taken from a token-order tensor: dst is that rank's
+ * rank-local rows [per_rank_actual_token[rank], row_bytes] (prev blocks of
+ * every sequence, then next blocks), src is [T, row_bytes].  This is the
+ * take-back that follows a reduction done in token order: each rank keeps its
+ * own zigzag rows, picked by token position rather than by rank-major row
+ * blocks (sgl-project/sglang pull request #39724, the CP-TP group sharing
+ * commit on token-order moves).  ZZ_ERR_INVALID_ARG if rank is outside
+ * [0, cp_size).  Same row/alignment rules as zz_shard_rows.
+ */
+zz_status_t zz_take_back_rows(const zz_plan_t* plan, int rank, const void* src, void* dst,
+                              int64_t row_bytes, void* stream);
 
 /*
  * Rerange the all-gathered K and V into the paged pool, in one pass
@@ -152,6 +177,22 @@ zz_status_t zz_rerange_kv_to_pool(const zz_plan_t* plan, const void* k_gathered,
                                   const void* v_gathered, void* k_pool, void* v_pool,
                                   const int64_t* out_cache_loc, int64_t num_slots,
                                   int h_kv, int d, zz_dtype_t dtype, void* stream);
+
+/*
+ * zz_rerange_kv_to_pool into an FP8 (E4M3, no infinities, max 448) pool with
+ * per-tensor scales (zigzag.py, materialize_full_kv passes layer.k_scale and
+ * layer.v_scale to set_kv_buffer):
+ *     k_pool[out_cache_loc[t]] = e4m3(k_gathered[src_row[t]] / k_scale)
+ * and the same for V.  The division is rounded in fp32; the conversion rounds
+ * to nearest even and saturates finite overflow to +-448; NaN stays NaN.
+ *   k_gathered, v_gathered: [c*M, h_kv, d] bf16; k_pool, v_pool: [num_slots,
+ *   h_kv, d] bytes.  h_kv*d a multiple of 16; scales positive and finite.
+ * v_gathered/v_pool may both be NULL.  Slots outside [0, num_slots) are skipped.
+ */
+zz_status_t zz_rerange_kv_to_pool_fp8(const zz_plan_t* plan, const void* k_gathered,
+                                      const void* v_gathered, void* k_pool, void* v_pool,
+                                      const int64_t* out_cache_loc, int64_t num_slots,
+                                      int h_kv, int d, float k_scale, float v_scale, void* stream);
 
 /*
  * Zigzag prefill attention for ranks [rank_begin, rank_begin + rank_count)

@@ -95,3 +95,62 @@ def test_rerange_k_only_and_out_of_range_slots_skipped():
     keep = [t for t in range(64) if t not in (5, 6)]
     assert np.array_equal(got[keep], nat[keep])
     assert (got[5] == 0).all() and (got[6] == 0).all()
+
+
+@pytest.mark.parametrize("cp,lens,width,dtype", [(4, [37, 50, 8], 16, torch.int32),
+                                                 (3, [300, 129], 1, torch.int32),   # 4-byte rows
+                                                 (2, [64, 90], 3, torch.int32),     # 12-byte rows
+                                                 (8, [4096], 2, torch.int64)])
+def test_gather_and_take_back_bit_exact(cp, lens, width, dtype):
+    ref = OP.build_metadata(cp, sum(lens), extend_lens=lens)
+    plan = zz.Plan(cp, extend_lens=lens)
+    plan.upload()
+    T = sum(lens)
+    x = (torch.arange(T * width, dtype=torch.int64).reshape(T, width) * 7 + 3).to(dtype)
+    xr = x if width > 1 else x.reshape(T)
+    ranked = torch.full((cp * plan.M,) + tuple(xr.shape[1:]), -1, dtype=dtype, device="cuda")
+    zz.shard_rows(plan, xr.cuda(), ranked)
+    want_ranked = OR.ranked_layout(xr.numpy(), ref)
+    got = ranked.cpu().numpy()
+    for r, n in enumerate(ref.per_rank_actual_token):
+        assert np.array_equal(got[r * ref.M: r * ref.M + n], want_ranked[r * ref.M: r * ref.M + n])
+    back = torch.full_like(xr.cuda(), -1)
+    zz.gather_rows(plan, ranked, back)          # gather_hidden_states
+    torch.cuda.synchronize()
+    assert np.array_equal(back.cpu().numpy(), OR.gather_kv(want_ranked, ref))
+    for r in range(cp):
+        mine = torch.full((ref.per_rank_actual_token[r],) + tuple(xr.shape[1:]), -1, dtype=dtype,
+                          device="cuda")
+        zz.take_back_rows(plan, r, xr.cuda(), mine)
+        torch.cuda.synchronize()
+        assert np.array_equal(mine.cpu().numpy(), OR.shard(xr.numpy(), ref, r))
+    with pytest.raises(zz.ZZError):
+        zz.take_back_rows(plan, cp, xr.cuda(), back)
+
+
+@pytest.mark.parametrize("cp,lens,h_kv,d,ks,vs", [(4, [4096], 4, 128, 0.37, 2.5),
+                                                  (3, [37, 1000, 129], 1, 64, 1e-3, 7.0),   # saturating K
+                                                  (8, [32768], 8, 128, 0.05, 0.05)])
+def test_rerange_fp8_pool_bit_exact(cp, lens, h_kv, d, ks, vs):
+    from oracle import fp8
+    ref = OP.build_metadata(cp, sum(lens), extend_lens=lens)
+    plan = zz.Plan(cp, extend_lens=lens)
+    plan.upload()
+    T = sum(lens)
+    _, k, v = synth.qkv(T, 1, h_kv, d, seed=9, scale=0.5, dtype="bf16", device="cpu")
+    pool = synth.paged_pool(lens, 16, seed=2, spare_pages=1)
+    kg = OR.ranked_layout(k.float().numpy(), ref)
+    vg = OR.ranked_layout(v.float().numpy(), ref)
+    kg_d = torch.from_numpy(kg).to(torch.bfloat16).cuda()   # exact: values are bf16 already
+    vg_d = torch.from_numpy(vg).to(torch.bfloat16).cuda()
+    kp = torch.full((pool.num_slots, h_kv, d), 0x55, dtype=torch.uint8, device="cuda")
+    vp = torch.full_like(kp, 0x55)
+    zz.rerange_kv_to_pool_fp8(plan, kg_d, vg_d, kp, vp, torch.from_numpy(pool.out_cache_loc).cuda(), ks, vs)
+    torch.cuda.synchronize()
+    base = np.full((pool.num_slots, h_kv, d), 0x55, np.uint8)
+    want_k = base.copy()
+    want_k[pool.out_cache_loc] = fp8.scale_encode(OR.gather_kv(kg, ref), ks)
+    want_v = base.copy()
+    want_v[pool.out_cache_loc] = fp8.scale_encode(OR.gather_kv(vg, ref), vs)
+    assert np.array_equal(kp.cpu().numpy(), want_k)
+    assert np.array_equal(vp.cpu().numpy(), want_v)

@@ -73,8 +73,12 @@ _sig = {
     "zz_plan_upload": (ctypes.c_int, [_P, _P, ctypes.c_size_t, _P]),
     "zz_plan_device_status": (ctypes.c_int, [_P, _I32P, ctypes.c_int, _P]),
     "zz_shard_rows": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P]),
+    "zz_gather_rows": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P]),
+    "zz_take_back_rows": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, ctypes.c_int64, _P]),
     "zz_rerange_kv_to_pool": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int64, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_int, _P]),
+    "zz_rerange_kv_to_pool_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int64, ctypes.c_int,
+                                                 ctypes.c_int, ctypes.c_float, ctypes.c_float, _P]),
     "zz_attn_prefill": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P, ctypes.c_int64,
                                        _P, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int, _P]),
@@ -199,6 +203,19 @@ def shard_rows(plan: Plan, src: torch.Tensor, dst: torch.Tensor, stream=None) ->
     _check(_lib.zz_shard_rows(plan.handle, _ptr(src), _ptr(dst), row_bytes, _stream(stream)))
 
 
+def gather_rows(plan: Plan, src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    """``dst[t] = src[src_row[t]]``: rank-ordered padded rows -> natural order."""
+    row_bytes = src[0].numel() * src.element_size()
+    _check(_lib.zz_gather_rows(plan.handle, _ptr(src), _ptr(dst), row_bytes, _stream(stream)))
+
+
+def take_back_rows(plan: Plan, rank: int, src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    """Rank ``rank``'s rank-local rows out of a natural-order tensor."""
+    row_bytes = src[0].numel() * src.element_size()
+    _check(_lib.zz_take_back_rows(plan.handle, int(rank), _ptr(src), _ptr(dst), row_bytes,
+                                  _stream(stream)))
+
+
 def rerange_kv_to_pool(plan: Plan, k_gathered, v_gathered, k_pool, v_pool, out_cache_loc,
                        stream=None) -> None:
     """Fused trim + rerange + pool write of the all-gathered K (and V)."""
@@ -206,6 +223,15 @@ def rerange_kv_to_pool(plan: Plan, k_gathered, v_gathered, k_pool, v_pool, out_c
     _check(_lib.zz_rerange_kv_to_pool(plan.handle, _ptr(k_gathered), _ptr(v_gathered), _ptr(k_pool),
                                       _ptr(v_pool), _ptr(out_cache_loc), k_pool.shape[0], h_kv, d,
                                       _DT[k_gathered.dtype], _stream(stream)))
+
+
+def rerange_kv_to_pool_fp8(plan: Plan, k_gathered, v_gathered, k_pool, v_pool, out_cache_loc,
+                           k_scale: float, v_scale: float = 1.0, stream=None) -> None:
+    """Fused rerange of bf16 K (and V) into E4M3 pools: ``e4m3(x / scale)``."""
+    h_kv, d = k_gathered.shape[-2], k_gathered.shape[-1]
+    _check(_lib.zz_rerange_kv_to_pool_fp8(plan.handle, _ptr(k_gathered), _ptr(v_gathered), _ptr(k_pool),
+                                          _ptr(v_pool), _ptr(out_cache_loc), k_pool.shape[0], h_kv, d,
+                                          float(k_scale), float(v_scale), _stream(stream)))
 
 
 def attn_prefill(plan: Plan, q, k_pool, v_pool, page_table, page_size: int, out, lse=None,

@@ -1,5 +1,5 @@
-// Row movement kernels: the fused K/V rerange into the paged pool, and the
-// natural -> rank-ordered shard.  Pure data movement, bound by HBM bandwidth.
+// The fused K/V rerange into the paged pool.  Pure data movement, bound by
+// HBM bandwidth.  (Token-order shard / gather / take-back live in permute.cu.)
 //
 // rerange (page "sgl-project--sglang/python/sglang/srt/layers/cp/zigzag.py",
 // _all_gather_reorganized + gather_kv_cache + materialize_full_kv): the page
@@ -110,7 +110,6 @@ zz_status_t launch_move(const MoveArgs& a, cudaStream_t s) {
   if (need < blocks) blocks = need;
   const unsigned b = unsigned(blocks);
   if (a.src_idx && a.dst_idx64) launch_kind<true, kDstI64>(a, b, s);        // rerange into the pool
-  else if (!a.src_idx && a.dst_idx32) launch_kind<false, kDstI32>(a, b, s);  // shard
   else return zz::fail(ZZ_ERR_INVALID_ARG, "move_rows: unsupported index maps");
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return zz::fail(ZZ_ERR_CUDA, std::string("move_rows launch: ") + cudaGetErrorString(e));
@@ -127,27 +126,6 @@ int pow2_shift(int64_t x) {
 }
 
 }  // namespace
-
-extern "C" zz_status_t zz_shard_rows(const zz_plan_t* plan, const void* src, void* dst,
-                                     int64_t row_bytes, void* stream) {
-  if (!plan || !src || !dst) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_shard_rows: NULL argument");
-  if (!plan->dev_ws) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_shard_rows: plan not uploaded");
-  if (row_bytes <= 0 || row_bytes % 16)
-    return zz::fail(ZZ_ERR_INVALID_ARG, "zz_shard_rows: row_bytes must be a positive multiple of 16");
-  if (!aligned16(src) || !aligned16(dst))
-    return zz::fail(ZZ_ERR_INVALID_ARG, "zz_shard_rows: pointers must be 16-byte aligned");
-  MoveArgs a{};
-  a.src[0] = static_cast<const int4*>(src);
-  a.dst[0] = static_cast<int4*>(dst);
-  a.src_idx = nullptr;
-  a.dst_idx32 = reinterpret_cast<const int32_t*>(static_cast<const char*>(plan->dev_ws) + plan->ws.src_row);
-  a.rows = plan->T;
-  a.vecs_per_row = row_bytes / 16;
-  a.vec_shift = pow2_shift(a.vecs_per_row);
-  a.ntensors = 1;
-  a.dst_rows = int64_t(plan->c) * plan->M;
-  return launch_move(a, static_cast<cudaStream_t>(stream));
-}
 
 extern "C" zz_status_t zz_rerange_kv_to_pool(const zz_plan_t* plan, const void* k_gathered,
                                              const void* v_gathered, void* k_pool, void* v_pool,

@@ -234,6 +234,24 @@ zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_coun
  */
 zz_status_t zz_debug_wait_timeout(int64_t timeout_ns, int64_t* dev_status, void* stream);
 
+/* Flags of zz_attn_prefill_ex. */
+enum { ZZ_ATTN_NONCAUSAL = 1 };
+
+/*
+ * zz_attn_prefill with flags.  ZZ_ATTN_NONCAUSAL drops the causal mask: every
+ * query row of a half attends to all keys of its sequence, prefix included
+ * (kv_len_next of rank 0, i.e. prefix + the whole extend length).  This is
+ * the local-Q / global-KV attention of an AllGather-KV layout, which is
+ * non-causal ("Compose Ulysses with AllGather-KV as a 2D SP topology",
+ * vllm-omni pull request #7937: local Q against the gathered global K/V).
+ * flags = 0 is exactly zz_attn_prefill.  Unknown flag bits: ZZ_ERR_INVALID_ARG.
+ */
+zz_status_t zz_attn_prefill_ex(const zz_plan_t* plan, int rank_begin, int rank_count,
+                               const void* q, const void* k_pool, const void* v_pool,
+                               int64_t num_slots, const int32_t* page_table, int max_pages,
+                               int page_size, void* out, float* lse, int h_q, int h_kv, int d,
+                               float softmax_scale, zz_dtype_t dtype, uint32_t flags, void* stream);
+
 /*
  * zz_attn_prefill without a workspace (bf16 only).  The zigzag pages have no
  * counterpart to this call; it exists for callers that cannot hand the library

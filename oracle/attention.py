@@ -38,18 +38,21 @@ def _as64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def attention_rows(q_rows, rows, k, v, kv_len: int, lq: int, scale: float):
+def attention_rows(q_rows, rows, k, v, kv_len: int, lq: int, scale: float, causal: bool = True):
     """Output and log-sum-exp of selected query rows of one half.
 
     ``q_rows``: ``[n, H_q, D]`` the queries of half-local rows ``rows``;
     ``k``, ``v``: ``[>= kv_len, H_kv, D]`` the sequence's keys and values in
     natural order.  Returns ``o [n, H_q, D]`` and ``lse [n, H_q]`` (natural log).
+    With ``causal=False`` every row sees all ``kv_len`` keys (the local-Q /
+    global-KV attention of an AllGather-KV layout, "Compose Ulysses with
+    AllGather-KV as a 2D SP topology": non-causal only).
     """
     q_rows, k, v = _as64(q_rows), _as64(k)[:kv_len], _as64(v)[:kv_len]
     n, h_q, d = q_rows.shape
     g = check_heads(h_q, k.shape[1])
     rows = np.asarray(rows, dtype=np.int64)
-    last_key = kv_len - lq + rows                           # inclusive
+    last_key = kv_len - lq + rows if causal else np.full(rows.shape, kv_len - 1)  # inclusive
     keys = np.arange(kv_len)
     visible = keys[None, :] <= last_key[:, None]            # [n, kv_len]
     o = np.empty((n, h_q, d))
@@ -66,24 +69,25 @@ def attention_rows(q_rows, rows, k, v, kv_len: int, lq: int, scale: float):
     return o, lse
 
 
-def attention_half(q_half, k, v, kv_len: int, scale: float, row_chunk: int = 512):
+def attention_half(q_half, k, v, kv_len: int, scale: float, row_chunk: int = 512, causal: bool = True):
     """All rows of one half (``Lq = q_half.shape[0]``), in row chunks."""
     lq = q_half.shape[0]
     outs, lses = [], []
     for a in range(0, lq, row_chunk):
         rows = np.arange(a, min(a + row_chunk, lq))
-        o, l = attention_rows(q_half[a:a + row_chunk], rows, k, v, kv_len, lq, scale)
+        o, l = attention_rows(q_half[a:a + row_chunk], rows, k, v, kv_len, lq, scale, causal)
         outs.append(o)
         lses.append(l)
     return np.concatenate(outs, 0), np.concatenate(lses, 0)
 
 
-def run_rank(plan: Plan, rank: int, q_local, k_seqs, v_seqs, scale: float):
+def run_rank(plan: Plan, rank: int, q_local, k_seqs, v_seqs, scale: float, causal: bool = True):
     """One rank's ``run_attention``: prev half then next half, concatenated.
 
     ``q_local``: ``[per_rank_actual_token[rank], H_q, D]`` rank-local queries;
     ``k_seqs[s]``/``v_seqs[s]``: full keys/values of sequence ``s`` (prefix
     included) in natural order.  Returns ``o`` and ``lse`` in rank-local order.
+    Non-causal: every half sees the whole sequence (prefix + extend keys).
     """
     q_local = _as64(q_local)
     split = plan.total_q_prev[rank]
@@ -92,7 +96,8 @@ def run_rank(plan: Plan, rank: int, q_local, k_seqs, v_seqs, scale: float):
     outs, lses = [], []
     for q_h, cu, kv_len in halves:
         for s in range(plan.bs):
-            o, l = attention_half(q_h[cu[s]:cu[s + 1]], k_seqs[s], v_seqs[s], kv_len[s], scale)
+            kv = kv_len[s] if causal else plan.prefix[s] + plan.extend_lens[s]
+            o, l = attention_half(q_h[cu[s]:cu[s + 1]], k_seqs[s], v_seqs[s], kv, scale, causal=causal)
             outs.append(o)
             lses.append(l)
     return np.concatenate(outs, 0), np.concatenate(lses, 0)
@@ -104,7 +109,7 @@ def full_causal(q_seq, k_seq, v_seq, scale: float):
     return attention_half(q_seq, k_seq, v_seq, _as64(k_seq).shape[0], scale)
 
 
-def brute_force(q_half, k, v, kv_len: int, scale: float):
+def brute_force(q_half, k, v, kv_len: int, scale: float, causal: bool = True):
     """Scalar restatement for tiny inputs: ``sum_j e^{s_j} v_j / sum_j e^{s_j}``
     over the visible keys, with ``math.exp`` and ``math.fsum``."""
     q_half, k, v = _as64(q_half).tolist(), _as64(k).tolist(), _as64(v).tolist()
@@ -112,7 +117,7 @@ def brute_force(q_half, k, v, kv_len: int, scale: float):
     g = h_q // len(k[0])
     out = [[[0.0] * d for _ in range(h_q)] for _ in range(lq)]
     for i in range(lq):
-        last = kv_len - lq + i
+        last = kv_len - lq + i if causal else kv_len - 1
         for h in range(h_q):
             kvh = h // g
             sc = [scale * math.fsum(q_half[i][h][t] * k[j][kvh][t] for t in range(d))

@@ -38,6 +38,7 @@ class Case:
     scale: float = 0.5           # value scale of the N(0,1) draws
     page_seed: int | None = 1
     prefix: list | None = None   # cached-prefix tokens per sequence (already in the pool)
+    causal: bool = True
 
 
 class Run:
@@ -95,7 +96,7 @@ class Run:
     def attend(self, rank_begin=0, rank_count=None):
         zz.attn_prefill(self.plan, self.q_ranked, self.k_pool, self.v_pool, self.page_table,
                         self.case.page_size, self.out, self.lse, softmax_scale=self.softmax_scale,
-                        rank_begin=rank_begin, rank_count=rank_count)
+                        rank_begin=rank_begin, rank_count=rank_count, causal=self.case.causal)
         torch.cuda.synchronize()
 
     # ---------------- oracle side
@@ -105,7 +106,7 @@ class Run:
                       else self.q.cpu().double().numpy(), self.ref_plan, r)
         ks = [k.cpu().double().numpy() for k in self.k_seqs]
         vs = [v.cpu().double().numpy() for v in self.v_seqs]
-        return OA.run_rank(self.ref_plan, r, ql, ks, vs, self.softmax_scale)
+        return OA.run_rank(self.ref_plan, r, ql, ks, vs, self.softmax_scale, causal=self.case.causal)
 
     def sampled_rows(self, per_half: int, rng_seed: int = 0):
         """[(rank, local_row, half, seq, row_in_half)] — first, last and random rows of every half."""

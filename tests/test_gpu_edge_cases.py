@@ -56,3 +56,13 @@ def test_bounded_wait_gives_up_and_context_stays_usable():
     assert 40_000_000 <= ns < 2_000_000_000
     # the context still runs real work afterwards
     _check_full(Run(Case(2, [200], 4, 2, 128, page_size=16)))
+
+
+@pytest.mark.parametrize("case", [
+    Case(2, [300, 517], 8, 2, 128, page_size=16, causal=False),
+    Case(3, [700], 4, 4, 128, page_size=64, causal=False),              # row-pair mode
+    Case(2, [260, 300], 4, 2, 128, page_size=16, prefix=[100, 37], causal=False),
+    Case(2, [256], 4, 4, 64, dtype="fp32", page_size=256, scale=1.0, page_seed=None, causal=False),
+], ids=["gqa", "mha", "prefix", "fp32"])
+def test_noncausal_local_q_global_kv(case):
+    _check_full(Run(case))

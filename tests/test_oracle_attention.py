@@ -132,3 +132,30 @@ def test_flop_count_closed_form():
     L = 2 * c * B
     p = P.build_metadata(c, L, extend_lens=[L])
     assert A.plan_flops(p, h_q, d) == 4 * d * h_q * (L * (L + 1) // 2)
+
+
+def test_noncausal_brute_force_and_library_softmax():
+    from scipy.special import softmax
+    lq, kv_len, h_q, h_kv, d = 6, 17, 4, 2, 5
+    q = _rand((lq, h_q, d), 30)
+    k = _rand((kv_len, h_kv, d), 31)
+    v = _rand((kv_len, h_kv, d), 32)
+    o, _ = A.attention_half(q, k, v, kv_len, 0.4, causal=False)
+    assert np.abs(o - A.brute_force(q, k, v, kv_len, 0.4, causal=False)).max() < 1e-13
+    for h in range(h_q):
+        p = softmax(0.4 * q[:, h] @ k[:, h // 2].T, axis=1)
+        assert np.abs(o[:, h] - p @ v[:, h // 2]).max() < 1e-13
+
+
+def test_noncausal_union_equals_full_noncausal_attention():
+    c, lens, h_q, h_kv, d = 3, [40, 29], 4, 1, 8
+    p = P.build_metadata(c, sum(lens), extend_lens=lens)
+    q, k, v = _rand((sum(lens), h_q, d), 33), _rand((sum(lens), h_kv, d), 34), _rand((sum(lens), h_kv, d), 35)
+    starts = np.cumsum([0] + lens)
+    ks = [k[starts[s]:starts[s + 1]] for s in range(2)]
+    vs = [v[starts[s]:starts[s + 1]] for s in range(2)]
+    per_rank = [A.run_rank(p, r, R.shard(q, p, r), ks, vs, 0.3, causal=False)[0] for r in range(c)]
+    o_tok = R.gather_kv(R.all_gather_padded(per_rank, p), p)
+    ref = np.concatenate([A.attention_half(q[starts[s]:starts[s + 1]], ks[s], vs[s], lens[s], 0.3,
+                                           causal=False)[0] for s in range(2)])
+    assert np.abs(o_tok - ref).max() < 1e-12

@@ -22,8 +22,8 @@ def test_off_by_one_mask_is_caught_by_brute_force(monkeypatch):
     good = A.brute_force(q, k, v, kv_len, 0.5)
     real = A.attention_rows
 
-    def shifted(q_rows, rows, k_, v_, kv_len_, lq_, scale):     # sees one key too few
-        return real(q_rows, rows, k_, v_, kv_len_ - 1, lq_, scale)
+    def shifted(q_rows, rows, k_, v_, kv_len_, lq_, scale, causal=True):   # sees one key too few
+        return real(q_rows, rows, k_, v_, kv_len_ - 1, lq_, scale, causal)
     monkeypatch.setattr(A, "attention_rows", shifted)
     bad, _ = A.attention_half(q, k, v, kv_len, 0.5)
     assert np.abs(bad - good).max() > 1e-3

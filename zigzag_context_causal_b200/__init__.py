@@ -84,6 +84,7 @@ _sig = {
                                        ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int, _P]),
 }
 _sig["zz_attn_prefill_noalloc"] = _sig["zz_attn_prefill"]
+_sig["zz_attn_prefill_ex"] = (ctypes.c_int, _sig["zz_attn_prefill"][1][:-1] + [ctypes.c_uint32, _P])
 _sig["zz_debug_wait_timeout"] = (ctypes.c_int, [ctypes.c_int64, _P, _P])
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)
@@ -234,9 +235,12 @@ def rerange_kv_to_pool_fp8(plan: Plan, k_gathered, v_gathered, k_pool, v_pool, o
                                           float(k_scale), float(v_scale), _stream(stream)))
 
 
+ZZ_ATTN_NONCAUSAL = 1
+
+
 def attn_prefill(plan: Plan, q, k_pool, v_pool, page_table, page_size: int, out, lse=None,
                  softmax_scale: float = 0.0, rank_begin: int = 0, rank_count: int | None = None,
-                 stream=None) -> None:
+                 stream=None, causal: bool = True) -> None:
     """Both zigzag halves of ranks [rank_begin, rank_begin+rank_count) in one launch.
 
     ``q``/``out``: ``[rank_count*M, H_q, D]`` (or ``[rank_count, M, H_q, D]``),
@@ -246,10 +250,11 @@ def attn_prefill(plan: Plan, q, k_pool, v_pool, page_table, page_size: int, out,
         rank_count = plan.cp_size
     h_q, d = q.shape[-2], q.shape[-1]
     h_kv = k_pool.shape[-2]
-    _check(_lib.zz_attn_prefill(plan.handle, rank_begin, rank_count, _ptr(q), _ptr(k_pool),
-                                _ptr(v_pool), k_pool.shape[0], _ptr(page_table), page_table.shape[1],
-                                int(page_size), _ptr(out), _ptr(lse), h_q, h_kv, d,
-                                float(softmax_scale), _DT[q.dtype], _stream(stream)))
+    _check(_lib.zz_attn_prefill_ex(plan.handle, rank_begin, rank_count, _ptr(q), _ptr(k_pool),
+                                   _ptr(v_pool), k_pool.shape[0], _ptr(page_table), page_table.shape[1],
+                                   int(page_size), _ptr(out), _ptr(lse), h_q, h_kv, d,
+                                   float(softmax_scale), _DT[q.dtype], 0 if causal else ZZ_ATTN_NONCAUSAL,
+                                   _stream(stream)))
 
 
 def raw_call(name: str, *args) -> int:

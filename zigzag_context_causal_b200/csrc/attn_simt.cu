@@ -31,6 +31,7 @@ struct SimtArgs {
   int h_q, h_kv, group;
   int M, rank_begin;
   float scale;
+  int causal;
 };
 
 template <int D>
@@ -57,9 +58,12 @@ __global__ void __launch_bounds__(kTileM) attn_simt_kernel(SimtArgs a) {
 #pragma unroll
   for (int i = 0; i < D; ++i) o[i] = 0.f;
   float m = -CUDART_INF_F, l = 0.f;
-  const int my_last = hd.kv_pos0 + row;                      // inclusive key bound
+  // Inclusive last key of my row and of the CTA; without the causal mask every
+  // row sees the whole sequence (kv_full keys).
+  const int kv_end = a.causal ? hd.kv_len : hd.kv_full;
+  const int my_last = a.causal ? hd.kv_pos0 + row : hd.kv_full - 1;
   const int tile_last_row = min(q0 + kTileM, hd.lq) - 1;
-  const int cta_last = hd.kv_pos0 + tile_last_row;
+  const int cta_last = a.causal ? hd.kv_pos0 + tile_last_row : hd.kv_full - 1;
   const int32_t* pt = a.page_table + int64_t(hd.seq) * a.max_pages;
   for (int k0 = 0; k0 <= cta_last; k0 += kChunk) {
     __syncthreads();
@@ -67,7 +71,7 @@ __global__ void __launch_bounds__(kTileM) attn_simt_kernel(SimtArgs a) {
       const int j = e / D, x = e % D;
       const int key = k0 + j;
       float kx = 0.f, vx = 0.f;
-      if (key < hd.kv_len) {
+      if (key < kv_end) {
         const int64_t slot = int64_t(pt[key / a.page_size]) * a.page_size + key % a.page_size;
         if (slot >= 0 && slot < a.num_slots) {
           const int64_t off = (slot * a.h_kv + kvh) * D + x;
@@ -118,7 +122,7 @@ zz_status_t launch_attn_simt_fp32(const zz_plan_t* p, int rank_begin, int rank_c
                                   const void* q, const void* k_pool, const void* v_pool,
                                   int64_t num_slots, const int32_t* page_table, int max_pages,
                                   int page_size, void* out, float* lse, int h_q, int h_kv, int d,
-                                  float scale, cudaStream_t s) {
+                                  float scale, int causal, cudaStream_t s) {
   const char* ws = static_cast<const char*>(p->dev_ws);
   SimtArgs a{};
   a.q = static_cast<const float*>(q);
@@ -145,6 +149,7 @@ zz_status_t launch_attn_simt_fp32(const zz_plan_t* p, int rank_begin, int rank_c
   a.M = p->M;
   a.rank_begin = rank_begin;
   a.scale = scale;
+  a.causal = causal;
   const int64_t grid = n_items * h_q;
   if (grid == 0) return ZZ_OK;
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: grid too large");

@@ -48,7 +48,7 @@ zz_status_t launch_attn_simt_fp32(const zz_plan_t* p, int rank_begin, int rank_c
                                   const void* q, const void* k_pool, const void* v_pool,
                                   int64_t num_slots, const int32_t* page_table, int max_pages,
                                   int page_size, void* out, float* lse, int h_q, int h_kv, int d,
-                                  float scale, cudaStream_t s);
+                                  float scale, int causal, cudaStream_t s);
 
 namespace {
 
@@ -102,6 +102,7 @@ struct Params {
   int max_pages, page_size, box_rows;
   float scale_log2;
   uint64_t timeout_ns;
+  int causal;           // 0: every row of a half sees all kv_full keys of its sequence
 };
 
 struct Bars {
@@ -122,8 +123,9 @@ struct SubTile {
   int n;    // K/V tiles to visit (0 = empty sub-tile)
 };
 
-__device__ __forceinline__ int tiles_for(const HalfDesc& h, int q0) {
+__device__ __forceinline__ int tiles_for(const HalfDesc& h, int q0, int causal) {
   if (q0 >= h.lq) return 0;
+  if (!causal) return (h.kv_full + 127) / 128;
   const int last_row = min(q0 + 128, h.lq) - 1;
   return (h.kv_pos0 + last_row) / 128 + 1;
 }
@@ -167,8 +169,9 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     st[0] = {hg, (2 * w.tile) * 128, 0};
     st[1] = {hg, (2 * w.tile + 1) * 128, 0};
   }
-  st[0].n = tiles_for(hd, st[0].q0);
-  st[1].n = tiles_for(hd, st[1].q0);
+  st[0].n = tiles_for(hd, st[0].q0, p.causal);
+  st[1].n = tiles_for(hd, st[1].q0, p.causal);
+  const int kv_end = p.causal ? hd.kv_len : hd.kv_full;   // keys that exist for this half
   const int n_max = max(st[0].n, st[1].n);
   const int kv_head = st[0].head / p.group;
   const int64_t row_base = int64_t(hd.rank - p.rank_begin) * p.M + hd.row0;  // Q/O row of half row 0
@@ -243,13 +246,13 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // slot can reach the MMAs (0 * NaN would poison P.V).
         bool manual = false;
         for (int c = 0; c < chunks; ++c) {
-          if (key0 + (c + 1) * p.box_rows <= hd.kv_len) tma_bytes += p.box_rows * 128 * C::kBoxes;
+          if (key0 + (c + 1) * p.box_rows <= kv_end) tma_bytes += p.box_rows * 128 * C::kBoxes;
           else manual = true;
         }
         if (manual) {
           const int units_per_row = C::kBoxes * 8;
           for (int c = 0; c < chunks; ++c) {
-            if (key0 + (c + 1) * p.box_rows <= hd.kv_len) continue;
+            if (key0 + (c + 1) * p.box_rows <= kv_end) continue;
             const int r_lo = c * p.box_rows;
             for (int u = lane; u < p.box_rows * units_per_row; u += 32) {
               const int row = r_lo + u / units_per_row;
@@ -257,7 +260,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               const int b = rem >> 3, ch = rem & 7;
               const int key = key0 + row;
               int4 v = make_int4(0, 0, 0, 0);
-              if (key < hd.kv_len) {
+              if (key < kv_end) {
                 const int64_t slot_id = int64_t(__ldg(pt + key / p.page_size)) * p.page_size + key % p.page_size;
                 if (slot_id >= 0 && slot_id < p.num_slots)
                   v = __ldg(reinterpret_cast<const int4*>(pool + (slot_id * p.h_kv + kv_head) * D + b * 64 + ch * 8));
@@ -279,7 +282,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const int key0 = tile_j * 128;
           for (int c = 0; c < chunks; ++c) {
             const int kc = key0 + c * p.box_rows;
-            if (kc + p.box_rows > hd.kv_len) continue;
+            if (kc + p.box_rows > kv_end) continue;
             const int32_t slot0 = __ldg(pt + kc / p.page_size) * p.page_size + kc % p.page_size;
             for (int b = 0; b < C::kBoxes; ++b)
               tma_load_3d(tile + b * C::kBoxBytes + c * p.box_rows * 128, tm, &bars->kv_full[slot],
@@ -376,8 +379,10 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t t_s = tmem + lane_off + (g ? C::kColS1 : C::kColS0);
     const uint32_t t_o = tmem + lane_off + (g ? C::kColO1 : C::kColO0);
     const int q_row = me.q0 + r;
-    const int my_pos = hd.kv_pos0 + q_row;     // last visible key (inclusive)
-    const int first_pos = hd.kv_pos0 + me.q0;  // position of the sub-tile's first row
+    // Last visible key (inclusive) of my row and of the sub-tile's first row;
+    // without the causal mask every row sees the whole sequence.
+    const int my_pos = p.causal ? hd.kv_pos0 + q_row : hd.kv_full - 1;
+    const int first_pos = p.causal ? hd.kv_pos0 + me.q0 : hd.kv_full - 1;
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = me.n > 0;
     for (int j = 0; j < me.n && ok; ++j) {
@@ -540,7 +545,7 @@ template <int D>
 zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, const void* q,
                         const void* k_pool, const void* v_pool, int64_t num_slots,
                         const int32_t* page_table, int max_pages, int page_size, void* out,
-                        float* lse, int h_q, int h_kv, float scale, cudaStream_t stream) {
+                        float* lse, int h_q, int h_kv, float scale, int causal, cudaStream_t stream) {
   using C = Cfg<D>;
   if (zz_status_t e = get_encoder()) return e;
   const int box_rows = page_size >= 128 ? 128 : page_size;
@@ -572,6 +577,7 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
   p.box_rows = box_rows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = 1000000000ull;   // 1 s per wait
+  p.causal = causal;
   int64_t n_items;
   const bool all = rank_count == pl->c;
   if (p.pair_heads) {
@@ -698,6 +704,7 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   p.box_rows = box_rows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = 1000000000ull;
+  p.causal = 1;
   const int64_t grid = int64_t(n_items) * p.head_groups;
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: grid too large");
   p.n_items = int(n_items);
@@ -713,12 +720,15 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
 }  // namespace
 }  // namespace zz
 
-extern "C" zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_count,
-                                       const void* q, const void* k_pool, const void* v_pool,
-                                       int64_t num_slots, const int32_t* page_table, int max_pages,
-                                       int page_size, void* out, float* lse, int h_q, int h_kv, int d,
-                                       float softmax_scale, zz_dtype_t dtype, void* stream) {
+extern "C" zz_status_t zz_attn_prefill_ex(const zz_plan_t* plan, int rank_begin, int rank_count,
+                                          const void* q, const void* k_pool, const void* v_pool,
+                                          int64_t num_slots, const int32_t* page_table, int max_pages,
+                                          int page_size, void* out, float* lse, int h_q, int h_kv,
+                                          int d, float softmax_scale, zz_dtype_t dtype, uint32_t flags,
+                                          void* stream) {
   using namespace zz;
+  if (flags & ~uint32_t(ZZ_ATTN_NONCAUSAL)) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: unknown flags");
+  const int causal = (flags & ZZ_ATTN_NONCAUSAL) ? 0 : 1;
   if (!plan || !q || !k_pool || !v_pool || !page_table || !out)
     return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: NULL argument");
   if (h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0)
@@ -743,7 +753,7 @@ extern "C" zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, in
   auto s = static_cast<cudaStream_t>(stream);
   if (dtype == ZZ_FP32)
     return launch_attn_simt_fp32(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
-                                 max_pages, page_size, out, lse, h_q, h_kv, d, scale, s);
+                                 max_pages, page_size, out, lse, h_q, h_kv, d, scale, causal, s);
   if (dtype != ZZ_BF16) return fail(ZZ_ERR_UNSUPPORTED, "zz_attn_prefill: dtype must be bf16 or fp32");
   const bool ps_ok = page_size == 8 || page_size == 16 || page_size == 32 || page_size == 64 ||
                      page_size % 128 == 0;
@@ -751,9 +761,18 @@ extern "C" zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, in
     return fail(ZZ_ERR_UNSUPPORTED, "zz_attn_prefill: bf16 page_size must be 8, 16, 32, 64 or a multiple of 128");
   if (d == 128)
     return launch_bf16<128>(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
-                            max_pages, page_size, out, lse, h_q, h_kv, scale, s);
+                            max_pages, page_size, out, lse, h_q, h_kv, scale, causal, s);
   return launch_bf16<64>(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
-                         max_pages, page_size, out, lse, h_q, h_kv, scale, s);
+                         max_pages, page_size, out, lse, h_q, h_kv, scale, causal, s);
+}
+
+extern "C" zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_count,
+                                       const void* q, const void* k_pool, const void* v_pool,
+                                       int64_t num_slots, const int32_t* page_table, int max_pages,
+                                       int page_size, void* out, float* lse, int h_q, int h_kv, int d,
+                                       float softmax_scale, zz_dtype_t dtype, void* stream) {
+  return zz_attn_prefill_ex(plan, rank_begin, rank_count, q, k_pool, v_pool, num_slots, page_table,
+                            max_pages, page_size, out, lse, h_q, h_kv, d, softmax_scale, dtype, 0u, stream);
 }
 
 // Allocation-free variant of zz_attn_prefill (bf16): same arguments, but the

@@ -23,7 +23,7 @@ struct HalfDesc {
   int32_t seq;        // sequence index (page-table row)
   int32_t kv_pos0;    // position of query row 0 = kv_len - lq
   int32_t half;       // 0 = prev, 1 = next
-  int32_t pad_;
+  int32_t kv_full;    // prefix + whole extend length: the keys a non-causal half sees
 };
 
 // One unit of attention work: rows [tile*128, tile*128+128) of a half, or for

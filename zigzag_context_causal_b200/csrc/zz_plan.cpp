@@ -64,6 +64,7 @@ static void build_tables(zz_plan* p) {
         d.kv_len = h == 0 ? p->kv_prev[r][s] : p->kv_next[r][s];
         d.row0 = h == 0 ? p->cu_prev[r][s] : p->total_prev[r] + p->cu_next[r][s];
         d.kv_pos0 = d.kv_len - d.lq;
+        d.kv_full = p->prefix[s] + p->ext[s];
         p->halves[(size_t(r) * 2 + h) * bs + s] = d;
       }
   // ---- longest-first work lists ----

@@ -73,6 +73,44 @@ def all_gather_rows(dist, out, local):
         dist.all_gather(list(out.chunk(dist.get_world_size())), local)
 
 
+def exchange_pools(dist, export, import_, pools, rank: int, world: int):
+    """Every rank's pools in rank order, as this GPU sees them.
+
+    ``pools``: this process's pool tensors (K, V).  ``export(t) -> (handle,
+    offset)`` names a tensor's allocation for other processes;
+    ``import_(handle, 0)`` maps a peer's whole allocation and returns an object
+    with ``.ptr`` (its start) and ``.close()``.  Two pools in one allocation
+    share one mapping.  Returns ``dsts[i][j]`` (tensor ``i`` of rank ``j``: the
+    tensor itself for this rank, a mapped address for the others) and the
+    mappings to close."""
+    mine = [export(p) for p in pools]
+    every = [None] * world
+    dist.all_gather_object(every, mine)
+    dsts = [[None] * world for _ in pools]
+    mapped, by_handle = [], {}
+    for j in range(world):
+        for i, p in enumerate(pools):
+            if j == rank:
+                dsts[i][j] = p
+                continue
+            handle, offset = every[j][i]
+            key = (j, bytes(handle))
+            if key not in by_handle:
+                by_handle[key] = import_(handle, 0)
+                mapped.append(by_handle[key])
+            dsts[i][j] = by_handle[key].ptr + offset
+    return dsts, mapped
+
+
+def push_all_local(zz, plan, r0: int, r_per: int, M: int, k_local, v_local, dsts, loc, num_slots: int):
+    """Push-form exchange: each virtual rank this process owns writes its K/V
+    rows into every process's pool (``dsts`` from ``exchange_pools``)."""
+    for vr in range(r0, r0 + r_per):
+        a, b = (vr - r0) * M, (vr - r0 + 1) * M
+        zz.rerange_push_kv(plan, vr, k_local[a:b], v_local[a:b], dsts[0], dsts[1],
+                           [loc] * len(dsts[0]), num_slots)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -274,16 +312,29 @@ def main_gpu(args):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     attn_ms, rr_ms = [], []
+    push = args.kv_exchange == "push"
+    mapped = []
+    if push:
+        if world > 1:
+            dsts, mapped = exchange_pools(dist, zz.ipc_export, zz.PeerBuffer, [k_pool, v_pool], rank, world)
+            fence_t = torch.zeros(1, device=dev)
+        else:
+            dsts = [[k_pool], [v_pool]]
 
     def step(record: bool):
         # S1 plan tables, S3 (multi-GPU only) all-gather, S4 rerange, S5 attention
         plan.upload(ws)
-        if world > 1:
+        if world > 1 and not push:
             all_gather_rows(dist, k_g, k_local)
             all_gather_rows(dist, v_g, v_local)
         e0, e1, e2 = ev(), ev(), ev()
         e0.record(stream)
-        zz.rerange_kv_to_pool(plan, k_g, v_g, k_pool, v_pool, loc)
+        if push:
+            push_all_local(zz, plan, r0, r_per, M, k_local, v_local, dsts, loc, pool.num_slots)
+            if world > 1:   # stream-ordered: every rank's pushes done before anyone's attention
+                dist.all_reduce(fence_t)
+        else:
+            zz.rerange_kv_to_pool(plan, k_g, v_g, k_pool, v_pool, loc)
         e1.record(stream)
         zz.attn_prefill(plan, q_mine, k_pool, v_pool, page_table, ps, out, softmax_scale=scale,
                         rank_begin=r0, rank_count=r_per)
@@ -332,19 +383,24 @@ def main_gpu(args):
         v_h.copy_(v_local)
         q_d = torch.empty_like(q_mine)
         # one GPU: its shard is the whole gathered buffer, copied straight into it
-        k_d = torch.empty_like(k_local) if world > 1 else k_g
-        v_d = torch.empty_like(v_local) if world > 1 else v_g
+        k_d = torch.empty_like(k_local) if world > 1 or push else k_g
+        v_d = torch.empty_like(v_local) if world > 1 or push else v_g
         e2e_steps = max(1, min(args.steps, 3))
 
         def e2e_step():
             q_d.copy_(q_h, non_blocking=True)
             k_d.copy_(k_h, non_blocking=True)
             v_d.copy_(v_h, non_blocking=True)
-            if world > 1:
-                all_gather_rows(dist, k_g, k_d)
-                all_gather_rows(dist, v_g, v_d)
             plan.upload(ws)
-            zz.rerange_kv_to_pool(plan, k_g, v_g, k_pool, v_pool, loc)
+            if push:
+                push_all_local(zz, plan, r0, r_per, M, k_d, v_d, dsts, loc, pool.num_slots)
+                if world > 1:
+                    dist.all_reduce(fence_t)
+            else:
+                if world > 1:
+                    all_gather_rows(dist, k_g, k_d)
+                    all_gather_rows(dist, v_g, v_d)
+                zz.rerange_kv_to_pool(plan, k_g, v_g, k_pool, v_pool, loc)
             zz.attn_prefill(plan, q_d, k_pool, v_pool, page_table, ps, out, softmax_scale=scale,
                             rank_begin=r0, rank_count=r_per)
             o_h.copy_(out, non_blocking=True)
@@ -375,6 +431,10 @@ def main_gpu(args):
         rerange_sweep = rerange_standalone(torch, zz, synth, dev)
 
     if world > 1:
+        dist.barrier()
+    if mapped:   # unmap peers' pools only once every rank is done writing into them
+        for m in mapped:
+            m.close()
         dist.barrier()
     if rank != 0:
         if world > 1:
@@ -407,6 +467,7 @@ def main_gpu(args):
         "config": {"workload": desc, "cp_size": cp, "seq_lens": lens if len(lens) <= 8 else len(lens),
                    "h_q": h_q, "h_kv": h_kv, "head_dim": d, "page_size": ps,
                    "parallelism": f"zigzag-cp{cp} (virtual ranks {r_per}/GPU)",
+                   "kv_exchange": args.kv_exchange,
                    "l2": "no flush: Q 2 GiB, gathered K/V 2x256 MiB and pool exceed the 126 MB L2"
                    if args.workload == "long" else "inputs sized per workload"},
         "attn_kernel_ms": attn_kernel_ms, "attn_tflops": attn_tflops,
@@ -419,7 +480,7 @@ def main_gpu(args):
                      "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel runs inside a long step)",
                      "traffic": traffic},
         "e2e": e2e,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (1 + (r_per if push else 1)) * args.steps,
         "device_status": status,
         "clocks": clocks,
         "cpu_baseline": cpu,
@@ -540,6 +601,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rerange-sweep", action="store_true")
+    ap.add_argument("--kv-exchange", default="allgather", choices=["allgather", "push"],
+                    help="allgather: NCCL all-gather then the rerange kernel; push: every rank's "
+                         "kernel writes its rows straight into every rank's pool (IPC-mapped)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

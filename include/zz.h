@@ -194,6 +194,65 @@ zz_status_t zz_rerange_kv_to_pool_fp8(const zz_plan_t* plan, const void* k_gathe
                                       const int64_t* out_cache_loc, int64_t num_slots,
                                       int h_kv, int d, float k_scale, float v_scale, void* stream);
 
+/* Most destination pools one zz_rerange_push_kv call writes. */
+enum { ZZ_MAX_PUSH_DST = 16 };
+
+/*
+ * All-gather and rerange fused, push style: rank `rank` writes its own K/V rows
+ * straight into the pool of every rank, so no gathered buffer and no separate
+ * rerange pass exist (zigzag.py, _all_gather_reorganized + materialize_full_kv:
+ * the all-gather of every rank's K/V followed by set_kv_buffer, with unit
+ * scales).  For every local row i < per_rank_actual_token[rank] holding
+ * natural token t, and every destination j < n_dst:
+ *     k_pools[j][out_cache_locs[j][t]] = k_local[i]
+ * and the same for V.
+ *   k_local, v_local: [>= per_rank_actual_token[rank], h_kv, d] this rank's
+ *     rank-local rows (prev blocks of every sequence, then next blocks), on the
+ *     calling GPU.
+ *   k_pools, v_pools: host arrays of n_dst device pointers, each a pool
+ *     [num_slots, h_kv, d] in the calling GPU's address space: its own pool or
+ *     a peer's pool mapped with zz_ipc_import (or peer access).  Stores to a
+ *     peer travel over NVLink as plain 16-byte stores; no TMA is used.
+ *   out_cache_locs: host array of n_dst device pointers to [T] int64 slot maps
+ *     readable by the calling GPU (one map may serve every destination).
+ * v_local and v_pools may both be NULL (one tensor).  1 <= n_dst <=
+ * ZZ_MAX_PUSH_DST.  Slots outside [0, num_slots) are skipped.  The call only
+ * enqueues the kernel: before any rank reads its pool, every rank's push into
+ * it must have completed (e.g. a stream-ordered collective or a host barrier
+ * after each rank's kernel).  Bit-exact copy; row h_kv*d*sizeof(dtype) a
+ * multiple of 16 bytes and every pointer 16-byte aligned.
+ * The pages gather first and rerange after; the push form is this library's
+ * own, and on one GPU it equals zz_rerange_kv_to_pool run per rank.
+ */
+zz_status_t zz_rerange_push_kv(const zz_plan_t* plan, int rank, const void* k_local,
+                               const void* v_local, void* const* k_pools, void* const* v_pools,
+                               const int64_t* const* out_cache_locs, int n_dst, int64_t num_slots,
+                               int h_kv, int d, zz_dtype_t dtype, void* stream);
+
+/* Bytes of an inter-process memory handle (cudaIpcMemHandle_t). */
+enum { ZZ_IPC_HANDLE_BYTES = 64 };
+
+/*
+ * Export a device buffer to other processes: `handle` (ZZ_IPC_HANDLE_BYTES,
+ * caller-owned host memory) names the allocation that contains dev_ptr and
+ * *offset is dev_ptr's distance from the allocation's start.  The allocation
+ * must come from cudaMalloc (as PyTorch's caching allocator does by default).
+ * No counterpart on the pages: it is how the push form reaches peers' pools.
+ */
+zz_status_t zz_ipc_export(const void* dev_ptr, void* handle, int64_t* offset);
+
+/*
+ * Map another process's exported buffer into this process: *base is the
+ * mapping of the whole allocation (pass it to zz_ipc_close), *dev_ptr =
+ * *base + offset.  Works between processes on the same GPU and between GPUs
+ * with peer access.  A handle exported by the calling process itself is
+ * rejected by CUDA (ZZ_ERR_CUDA).
+ */
+zz_status_t zz_ipc_import(const void* handle, int64_t offset, void** base, void** dev_ptr);
+
+/* Unmap a base returned by zz_ipc_import. */
+zz_status_t zz_ipc_close(void* base);
+
 /*
  * Zigzag prefill attention for ranks [rank_begin, rank_begin + rank_count)
  * in ONE launch (zigzag.py, run_attention: prev half then next half).  For

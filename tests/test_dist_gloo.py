@@ -76,3 +76,58 @@ def test_rank_range_rejects_uneven_split():
     import bench
     with pytest.raises(ValueError):
         bench.rank_range(6, 4, 0)
+
+
+class _FakeMap:
+    def __init__(self, handle, offset, log):
+        self.ptr = 1_000_000 * int(handle.decode().split(":")[1]) + offset
+        self.handle = handle
+        self.closed = False
+        log.append(handle)
+
+    def close(self):
+        self.closed = True
+
+
+def _exchange_worker(rank, world, port, out_q):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        import bench
+        # K and V of one rank share an allocation ("alloc:<rank>"), at offsets 0 and 4096
+        pools = ["K", "V"]
+        export = lambda t: (f"alloc:{rank + 1}".encode(), 0 if t == "K" else 4096)  # noqa: E731
+        log = []
+        dsts, mapped = bench.exchange_pools(dist, export, lambda h, o: _FakeMap(h, o, log), pools,
+                                            rank, world)
+        out_q.put((rank, dsts, [m.handle for m in mapped], log))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_exchange_pools_orders_destinations_by_rank():
+    """Destination j of the push is rank j's pool; this rank's own tensors stay
+    tensors; one mapping per peer allocation, shared by K and V."""
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_exchange_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=30)
+    for rank, dsts, mapped, log in res:
+        for j in range(world):
+            if j == rank:
+                assert dsts[0][j] == "K" and dsts[1][j] == "V"
+            else:
+                assert dsts[0][j] == 1_000_000 * (j + 1)
+                assert dsts[1][j] == 1_000_000 * (j + 1) + 4096
+        assert sorted(mapped) == sorted(f"alloc:{j + 1}".encode() for j in range(world) if j != rank)
+        assert len(log) == world - 1

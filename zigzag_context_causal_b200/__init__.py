@@ -86,6 +86,14 @@ _sig = {
 _sig["zz_attn_prefill_noalloc"] = _sig["zz_attn_prefill"]
 _sig["zz_attn_prefill_ex"] = (ctypes.c_int, _sig["zz_attn_prefill"][1][:-1] + [ctypes.c_uint32, _P])
 _sig["zz_debug_wait_timeout"] = (ctypes.c_int, [ctypes.c_int64, _P, _P])
+_PP = ctypes.POINTER(_P)
+_sig["zz_rerange_push_kv"] = (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _PP, _PP, _PP, ctypes.c_int,
+                                             ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P])
+_sig["zz_ipc_export"] = (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int64)])
+_sig["zz_ipc_import"] = (ctypes.c_int, [_P, ctypes.c_int64, _PP, _PP])
+_sig["zz_ipc_close"] = (ctypes.c_int, [_P])
+ZZ_MAX_PUSH_DST = 16
+ZZ_IPC_HANDLE_BYTES = 64
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
@@ -233,6 +241,55 @@ def rerange_kv_to_pool_fp8(plan: Plan, k_gathered, v_gathered, k_pool, v_pool, o
     _check(_lib.zz_rerange_kv_to_pool_fp8(plan.handle, _ptr(k_gathered), _ptr(v_gathered), _ptr(k_pool),
                                           _ptr(v_pool), _ptr(out_cache_loc), k_pool.shape[0], h_kv, d,
                                           float(k_scale), float(v_scale), _stream(stream)))
+
+
+def _addr(x) -> int:
+    """Device address of a tensor, or an int already holding one (a mapped peer buffer)."""
+    return x if isinstance(x, int) else _ptr(x)
+
+
+def rerange_push_kv(plan: Plan, rank: int, k_local, v_local, k_pools, v_pools, out_cache_locs,
+                    num_slots: int, stream=None) -> None:
+    """Rank ``rank`` writes its local K (and V) rows into every pool of the lists.
+
+    ``k_local``/``v_local``: ``[>= per_rank_actual_token[rank], H_kv, D]``;
+    ``k_pools``/``v_pools``/``out_cache_locs``: one entry per destination, each a
+    tensor on this GPU or an int address (a peer pool mapped with ``PeerBuffer``).
+    """
+    n = len(k_pools)
+    if v_pools is not None and len(v_pools) != n or len(out_cache_locs) != n:
+        raise ValueError("k_pools, v_pools and out_cache_locs must have one entry per destination")
+    kp = (_P * n)(*[_addr(x) for x in k_pools])
+    vp = (_P * n)(*[_addr(x) for x in v_pools]) if v_pools is not None else None
+    lp = (_P * n)(*[_addr(x) for x in out_cache_locs])
+    h_kv, d = k_local.shape[-2], k_local.shape[-1]
+    _check(_lib.zz_rerange_push_kv(plan.handle, int(rank), _ptr(k_local), _ptr(v_local), kp, vp, lp, n,
+                                   int(num_slots), h_kv, d, _DT[k_local.dtype], _stream(stream)))
+
+
+def ipc_export(t: torch.Tensor) -> tuple[bytes, int]:
+    """(handle, offset) naming ``t``'s device memory for another process."""
+    buf = ctypes.create_string_buffer(ZZ_IPC_HANDLE_BYTES)
+    off = ctypes.c_int64(0)
+    _check(_lib.zz_ipc_export(_ptr(t), buf, ctypes.byref(off)))
+    return buf.raw, off.value
+
+
+class PeerBuffer:
+    """Another process's exported buffer mapped into this one; ``ptr`` is its address."""
+
+    def __init__(self, handle: bytes, offset: int):
+        if len(handle) != ZZ_IPC_HANDLE_BYTES:
+            raise ValueError("IPC handle must be 64 bytes")
+        base, ptr = _P(), _P()
+        _check(_lib.zz_ipc_import(handle, int(offset), ctypes.byref(base), ctypes.byref(ptr)))
+        self._base = base.value
+        self.ptr = ptr.value
+
+    def close(self) -> None:
+        if self._base:
+            _check(_lib.zz_ipc_close(self._base))
+            self._base = None
 
 
 ZZ_ATTN_NONCAUSAL = 1

@@ -12,7 +12,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libzz.so")
-SOURCES = ["zz_plan.cpp", "rerange.cu", "rerange_fp8.cu", "permute.cu", "attn_simt.cu", "attn_sm100.cu", "selftest.cu"]
+SOURCES = ["zz_plan.cpp", "rerange.cu", "rerange_fp8.cu", "permute.cu", "push.cu", "attn_simt.cu", "attn_sm100.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -34,7 +34,7 @@ struct WorkItem {
 };
 
 struct Workspace {  // byte offsets into the device workspace
-  size_t src_row, halves, tiles_all, tiles_rank, pairs_all, pairs_rank, status, total;
+  size_t src_row, rank_tok, halves, tiles_all, tiles_rank, pairs_all, pairs_rank, status, total;
 };
 
 }  // namespace zz
@@ -51,6 +51,7 @@ struct zz_plan {
   std::vector<std::vector<int32_t>> cu_prev, cu_next;             // [c][bs+1]
   std::vector<int32_t> total_prev, total_next, max_q_prev, max_q_next;  // [c]
   std::vector<int32_t> src_row;                                   // [T]
+  std::vector<int32_t> rank_tok;                                  // [c*M]: inverse of src_row, -1 = pad
   int64_t causal_pairs = 0;
   // device tables, host copies
   std::vector<zz::HalfDesc> halves;                               // [c*2*bs]

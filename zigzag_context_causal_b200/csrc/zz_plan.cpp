@@ -51,6 +51,9 @@ static void build_tables(zz_plan* p) {
         p->src_row[t++] = int32_t(int64_t(r) * p->M + start + o);
     }
   }
+  // ---- rank-ordered row -> natural token (padding rows: -1) ----
+  p->rank_tok.assign(size_t(c) * p->M, -1);
+  for (int64_t i = 0; i < p->T; ++i) p->rank_tok[p->src_row[i]] = int32_t(i);
   // ---- half descriptors, id = (r*2 + half)*bs + s ----
   p->halves.assign(size_t(c) * 2 * bs, HalfDesc{});
   for (int r = 0; r < c; ++r)
@@ -113,6 +116,7 @@ static void build_tables(zz_plan* p) {
   zz::Workspace& w = p->ws;
   size_t at = 0;
   w.src_row = at;    at = align256(at + sizeof(int32_t) * size_t(p->T));
+  w.rank_tok = at;   at = align256(at + sizeof(int32_t) * p->rank_tok.size());
   w.halves = at;     at = align256(at + sizeof(HalfDesc) * p->halves.size());
   w.tiles_all = at;  at = align256(at + sizeof(WorkItem) * p->tiles_all.size());
   w.tiles_rank = at; at = align256(at + sizeof(WorkItem) * p->tiles_rank.size());
@@ -328,6 +332,7 @@ extern "C" zz_status_t zz_plan_upload(zz_plan_t* p, void* dev, size_t bytes, voi
   char* base = static_cast<char*>(dev);
   struct Part { size_t off; const void* src; size_t n; } parts[] = {
       {p->ws.src_row, p->src_row.data(), p->src_row.size() * sizeof(int32_t)},
+      {p->ws.rank_tok, p->rank_tok.data(), p->rank_tok.size() * sizeof(int32_t)},
       {p->ws.halves, p->halves.data(), p->halves.size() * sizeof(zz::HalfDesc)},
       {p->ws.tiles_all, p->tiles_all.data(), p->tiles_all.size() * sizeof(zz::WorkItem)},
       {p->ws.tiles_rank, p->tiles_rank.data(), p->tiles_rank.size() * sizeof(zz::WorkItem)},

@@ -120,9 +120,12 @@ zz_status_t zz_plan_upload(zz_plan_t* plan, void* dev_workspace, size_t bytes, v
 
 /*
  * Read (and optionally clear) the device status word that the kernels of this
- * plan set when a bounded device-side wait gives up instead of hanging.
- * Synchronises `stream` (a diagnostic, not a hot-path call).  Returns
- * ZZ_ERR_DEVICE_TIMEOUT when bit 0 of *flags is set, ZZ_OK otherwise.
+ * plan set: bit 0 (value 1) when a bounded device-side wait gave up instead of
+ * hanging, bit 2 (value 4) when the attention read a page_table entry that
+ * points outside the pool (those keys were read as zeros).  Synchronises
+ * `stream` (a diagnostic, not a hot-path call).  Returns ZZ_ERR_DEVICE_TIMEOUT
+ * when bit 0 is set, else ZZ_ERR_INVALID_ARG when bit 2 is set, else ZZ_OK.
+ * zz_plan_upload clears the word.
  */
 zz_status_t zz_plan_device_status(const zz_plan_t* plan, int32_t* flags, int clear, void* stream);
 
@@ -266,7 +269,9 @@ zz_status_t zz_ipc_close(void* base);
  *   k_pool, v_pool: [num_slots, h_kv, d]; page_table [bs, max_pages] int32;
  *           slot of key t of sequence s = page_table[s][t/page_size]*page_size
  *           + t%page_size.  Only the first ceil(kv_len/page_size) entries of a
- *           row are read.
+ *           row are read.  An entry whose slots fall outside [0, num_slots)
+ *           is not dereferenced: its keys read as zeros and bit 2 of the
+ *           plan's status word is set (see zz_plan_device_status).
  *   lse: optional [rank_count, M, h_q] fp32 natural-log sum of exponentials.
  *   softmax_scale <= 0 selects 1/sqrt(d).
  * Errors: ZZ_ERR_INVALID_ARG when h_q % h_kv != 0 (message names "multiple of

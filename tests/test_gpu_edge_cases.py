@@ -66,3 +66,28 @@ def test_bounded_wait_gives_up_and_context_stays_usable():
 ], ids=["gqa", "mha", "prefix", "fp32"])
 def test_noncausal_local_q_global_kv(case):
     _check_full(Run(case))
+
+
+@pytest.mark.parametrize("dtype,d,ps,bad", [("bf16", 128, 16, 10**6), ("bf16", 128, 64, -1),
+                                           ("fp32", 64, 256, 2**28)],
+                         ids=["bf16-past-end", "bf16-negative", "fp32-past-end"])
+def test_page_outside_pool_is_reported_and_contained(dtype, d, ps, bad):
+    """A page-table entry outside the pool is never dereferenced: its keys read as
+    zeros, the status word reports it, other sequences stay exact, and the
+    context keeps working."""
+    run = Run(Case(2, [300, 212], 4, 2, d, dtype=dtype, page_size=ps, scale=0.5))
+    run.page_table[0, 1] = bad                       # sequence 0, second page
+    run.attend()
+    with pytest.raises(zz.ZZError, match="outside the pool") as e:
+        run.plan.device_status()
+    assert e.value.status == zz.ZZ_ERR_INVALID_ARG
+    assert run.plan.device_status() == 0             # the read cleared it
+    p = run.ref_plan
+    out = run.out.float().cpu().numpy()
+    for r in range(p.cp_size):
+        o_ref, _ = run.expected_rank(r)
+        tp = p.total_q_prev[r]
+        for lo, hi in ((p.cu_seqlens_q_prev[r][1], p.cu_seqlens_q_prev[r][2]),
+                       (tp + p.cu_seqlens_q_next[r][1], tp + p.cu_seqlens_q_next[r][2])):
+            assert_close(out[r * p.M + lo: r * p.M + hi], o_ref[lo:hi], dtype, f"rank {r} seq 1")
+    _check_full(Run(Case(2, [200], 4, 2, 128, page_size=16)))

@@ -32,6 +32,7 @@ struct SimtArgs {
   int M, rank_begin;
   float scale;
   int causal;
+  int* status;          // device status word (kStatusBadPage)
 };
 
 template <int D>
@@ -65,6 +66,7 @@ __global__ void __launch_bounds__(kTileM) attn_simt_kernel(SimtArgs a) {
   const int tile_last_row = min(q0 + kTileM, hd.lq) - 1;
   const int cta_last = a.causal ? hd.kv_pos0 + tile_last_row : hd.kv_full - 1;
   const int32_t* pt = a.page_table + int64_t(hd.seq) * a.max_pages;
+  bool bad_page = false;   // a page outside the pool: its keys read as zeros, reported in status
   for (int k0 = 0; k0 <= cta_last; k0 += kChunk) {
     __syncthreads();
     for (int e = threadIdx.x; e < kChunk * D; e += blockDim.x) {
@@ -77,6 +79,8 @@ __global__ void __launch_bounds__(kTileM) attn_simt_kernel(SimtArgs a) {
           const int64_t off = (slot * a.h_kv + kvh) * D + x;
           kx = a.k_pool[off];
           vx = a.v_pool[off];
+        } else {
+          bad_page = true;
         }
       }
       ks[j][x] = kx;
@@ -108,6 +112,7 @@ __global__ void __launch_bounds__(kTileM) attn_simt_kernel(SimtArgs a) {
     }
     m = m_new;
   }
+  if (bad_page && a.status) atomicOr(a.status, kStatusBadPage);
   if (!valid) return;
   const float inv = 1.f / l;
   float* op = a.out + (grow * a.h_q + head) * D;
@@ -150,6 +155,7 @@ zz_status_t launch_attn_simt_fp32(const zz_plan_t* p, int rank_begin, int rank_c
   a.rank_begin = rank_begin;
   a.scale = scale;
   a.causal = causal;
+  a.status = reinterpret_cast<int*>(const_cast<char*>(ws) + p->ws.status);
   const int64_t grid = n_items * h_q;
   if (grid == 0) return ZZ_OK;
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: grid too large");

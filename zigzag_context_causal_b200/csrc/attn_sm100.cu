@@ -40,6 +40,7 @@
 
 #include "ptx_sm100.cuh"
 #include "exp2_poly.h"
+#include "nvtx_range.h"
 #include "zz_internal.h"
 
 namespace zz {
@@ -100,6 +101,7 @@ struct Params {
   int n_items;
   int M, rank_begin;
   int max_pages, page_size, box_rows;
+  int num_pages;        // ceil(num_slots / page_size): valid page ids are [0, num_pages)
   float scale_log2;
   uint64_t timeout_ns;
   int causal;           // 0: every row of a half sees all kv_full keys of its sequence
@@ -191,7 +193,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     // A CTA that timed out earlier in this launch (or an earlier launch of
     // this plan) has set the status word: skip the work instead of waiting.
-    bars->abort = (p.status && *reinterpret_cast<volatile int*>(p.status)) ? 1 : 0;
+    bars->abort = (p.status && (*reinterpret_cast<volatile int*>(p.status) & kStatusTimeout)) ? 1 : 0;
     fence_barrier_init();
   }
   if (warp == kWarpMma) {
@@ -227,6 +229,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
     }
     const int chunks = 128 / p.box_rows;
+    bool bad_page = false;
     // Stage t (t = 0 .. n_max): K_t if t < n_max, V_{t-1} if t >= 1.
     int t = 0;
     for (; t <= n_max && !*abort; ++t) {
@@ -264,6 +267,8 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int64_t slot_id = int64_t(__ldg(pt + key / p.page_size)) * p.page_size + key % p.page_size;
                 if (slot_id >= 0 && slot_id < p.num_slots)
                   v = __ldg(reinterpret_cast<const int4*>(pool + (slot_id * p.h_kv + kv_head) * D + b * 64 + ch * 8));
+                else
+                  bad_page = true;
               }
               *reinterpret_cast<int4*>(tile + b * C::kBoxBytes + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
             }
@@ -283,7 +288,12 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int c = 0; c < chunks; ++c) {
             const int kc = key0 + c * p.box_rows;
             if (kc + p.box_rows > kv_end) continue;
-            const int32_t slot0 = __ldg(pt + kc / p.page_size) * p.page_size + kc % p.page_size;
+            // A page outside the pool is loaded from a coordinate past the pool's
+            // end (zero fill) and reported through the status word.
+            const int32_t page = __ldg(pt + kc / p.page_size);
+            const bool in_pool = uint32_t(page) < uint32_t(p.num_pages);
+            bad_page |= !in_pool;
+            const int32_t slot0 = (in_pool ? page : p.num_pages) * p.page_size + kc % p.page_size;
             for (int b = 0; b < C::kBoxes; ++b)
               tma_load_3d(tile + b * C::kBoxBytes + c * p.box_rows * 128, tm, &bars->kv_full[slot],
                           b * 64, kv_head, slot0);
@@ -293,6 +303,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       __syncwarp();
     }
     const int load_no = t;   // stages issued
+    if (bad_page && p.status) atomicOr(p.status, kStatusBadPage);
     // Never leave with copies in flight into shared memory.
     if (lane == 0) {
       for (int n = max(0, load_no - C::kStages); n < load_no; ++n)
@@ -493,7 +504,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && bars->abort && p.status) {
-    atomicOr(p.status, 1);
+    atomicOr(p.status, kStatusTimeout);
     __threadfence();
   }
 }
@@ -575,6 +586,8 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
   p.max_pages = max_pages;
   p.page_size = page_size;
   p.box_rows = box_rows;
+  if (num_slots > int64_t(INT32_MAX) - page_size) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: num_slots too large");
+  p.num_pages = int((num_slots + page_size - 1) / page_size);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = 1000000000ull;   // 1 s per wait
   p.causal = causal;
@@ -702,6 +715,8 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   p.max_pages = max_pages;
   p.page_size = page_size;
   p.box_rows = box_rows;
+  if (num_slots > int64_t(INT32_MAX) - page_size) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: num_slots too large");
+  p.num_pages = int((num_slots + page_size - 1) / page_size);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = 1000000000ull;
   p.causal = 1;
@@ -726,6 +741,7 @@ extern "C" zz_status_t zz_attn_prefill_ex(const zz_plan_t* plan, int rank_begin,
                                           int page_size, void* out, float* lse, int h_q, int h_kv,
                                           int d, float softmax_scale, zz_dtype_t dtype, uint32_t flags,
                                           void* stream) {
+  ZZ_NVTX("zz_attn_prefill_ex");
   using namespace zz;
   if (flags & ~uint32_t(ZZ_ATTN_NONCAUSAL)) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: unknown flags");
   const int causal = (flags & ZZ_ATTN_NONCAUSAL) ? 0 : 1;
@@ -784,6 +800,7 @@ extern "C" zz_status_t zz_attn_prefill_noalloc(const zz_plan_t* plan, int rank_b
                                                int max_pages, int page_size, void* out, float* lse,
                                                int h_q, int h_kv, int d, float softmax_scale,
                                                zz_dtype_t dtype, void* stream) {
+  ZZ_NVTX("zz_attn_prefill_noalloc");
   using namespace zz;
   if (!plan || !q || !k_pool || !v_pool || !page_table || !out)
     return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: NULL argument");

@@ -8,6 +8,7 @@
 
 #include <string>
 
+#include "nvtx_range.h"
 #include "zz_internal.h"
 
 namespace {
@@ -99,6 +100,7 @@ zz_status_t launch_permute(const char* who, const zz_plan_t* plan, const void* s
 
 extern "C" zz_status_t zz_shard_rows(const zz_plan_t* plan, const void* src, void* dst,
                                      int64_t row_bytes, void* stream) {
+  ZZ_NVTX("zz_shard_rows");
   if (!plan) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_shard_rows: NULL plan");
   return launch_permute("zz_shard_rows", plan, src, dst, row_bytes, 0, 1, int64_t(plan->c) * plan->M,
                         static_cast<cudaStream_t>(stream));
@@ -106,6 +108,7 @@ extern "C" zz_status_t zz_shard_rows(const zz_plan_t* plan, const void* src, voi
 
 extern "C" zz_status_t zz_gather_rows(const zz_plan_t* plan, const void* src, void* dst,
                                       int64_t row_bytes, void* stream) {
+  ZZ_NVTX("zz_gather_rows");
   if (!plan) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_gather_rows: NULL plan");
   return launch_permute("zz_gather_rows", plan, src, dst, row_bytes, 0, 0, plan->T,
                         static_cast<cudaStream_t>(stream));
@@ -113,6 +116,7 @@ extern "C" zz_status_t zz_gather_rows(const zz_plan_t* plan, const void* src, vo
 
 extern "C" zz_status_t zz_take_back_rows(const zz_plan_t* plan, int rank, const void* src, void* dst,
                                          int64_t row_bytes, void* stream) {
+  ZZ_NVTX("zz_take_back_rows");
   if (!plan) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_take_back_rows: NULL plan");
   if (rank < 0 || rank >= plan->c) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_take_back_rows: rank out of range");
   return launch_permute("zz_take_back_rows", plan, src, dst, row_bytes, int64_t(rank) * plan->M, 1,

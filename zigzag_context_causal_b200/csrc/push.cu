@@ -19,6 +19,7 @@
 #include <mutex>
 #include <string>
 
+#include "nvtx_range.h"
 #include "zz_internal.h"
 
 namespace {
@@ -117,6 +118,7 @@ extern "C" zz_status_t zz_rerange_push_kv(const zz_plan_t* plan, int rank, const
                                           void* const* v_pools, const int64_t* const* out_cache_locs,
                                           int n_dst, int64_t num_slots, int h_kv, int d,
                                           zz_dtype_t dtype, void* stream) {
+  ZZ_NVTX("zz_rerange_push_kv");
   if (!plan || !k_local || !k_pools || !out_cache_locs)
     return zz::fail(ZZ_ERR_INVALID_ARG, "zz_rerange_push_kv: NULL argument");
   if ((v_local == nullptr) != (v_pools == nullptr))

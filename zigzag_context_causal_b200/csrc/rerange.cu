@@ -13,6 +13,7 @@
 
 #include <string>
 
+#include "nvtx_range.h"
 #include "zz_internal.h"
 
 namespace {
@@ -131,6 +132,7 @@ extern "C" zz_status_t zz_rerange_kv_to_pool(const zz_plan_t* plan, const void* 
                                              const void* v_gathered, void* k_pool, void* v_pool,
                                              const int64_t* out_cache_loc, int64_t num_slots,
                                              int h_kv, int d, zz_dtype_t dtype, void* stream) {
+  ZZ_NVTX("zz_rerange_kv_to_pool");
   if (!plan || !k_gathered || !k_pool || !out_cache_loc)
     return zz::fail(ZZ_ERR_INVALID_ARG, "zz_rerange_kv_to_pool: NULL argument");
   if ((v_gathered == nullptr) != (v_pool == nullptr))

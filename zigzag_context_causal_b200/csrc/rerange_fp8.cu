@@ -11,6 +11,7 @@
 #include <cmath>
 #include <string>
 
+#include "nvtx_range.h"
 #include "zz_internal.h"
 
 namespace {
@@ -94,6 +95,7 @@ extern "C" zz_status_t zz_rerange_kv_to_pool_fp8(const zz_plan_t* plan, const vo
                                                  const int64_t* out_cache_loc, int64_t num_slots,
                                                  int h_kv, int d, float k_scale, float v_scale,
                                                  void* stream) {
+  ZZ_NVTX("zz_rerange_kv_to_pool_fp8");
   if (!plan || !k_gathered || !k_pool || !out_cache_loc)
     return zz::fail(ZZ_ERR_INVALID_ARG, "zz_rerange_kv_to_pool_fp8: NULL argument");
   if ((v_gathered == nullptr) != (v_pool == nullptr))

@@ -5,6 +5,7 @@
 #include <string>
 
 #include "ptx_sm100.cuh"
+#include "nvtx_range.h"
 #include "zz_internal.h"
 
 using namespace zz::dev;
@@ -29,6 +30,7 @@ __global__ void wait_timeout_probe(uint64_t timeout_ns, int64_t* status) {
 }  // namespace zz
 
 extern "C" zz_status_t zz_debug_wait_timeout(int64_t timeout_ns, int64_t* dev_status, void* stream) {
+  ZZ_NVTX("zz_debug_wait_timeout");
   using namespace zz;
   if (!dev_status || timeout_ns <= 0 || timeout_ns > 10000000000ll)
     return fail(ZZ_ERR_INVALID_ARG, "zz_debug_wait_timeout: need dev_status and 0 < timeout_ns <= 10 s");

@@ -33,6 +33,10 @@ struct WorkItem {
   int32_t tile;
 };
 
+// Bits of the device status word (kernels OR them in; zz_plan_device_status reads them).
+constexpr int kStatusTimeout = 1;   // a bounded wait gave up
+constexpr int kStatusBadPage = 4;   // a page_table entry pointed outside the pool
+
 struct Workspace {  // byte offsets into the device workspace
   size_t src_row, rank_tok, halves, tiles_all, tiles_rank, pairs_all, pairs_rank, status, total;
 };

@@ -9,6 +9,7 @@
 
 #include <cuda_runtime.h>
 
+#include "nvtx_range.h"
 #include "zz_internal.h"
 
 namespace {
@@ -324,6 +325,7 @@ extern "C" zz_status_t zz_plan_get(const zz_plan_t* p, int rank, zz_field_t fiel
 extern "C" size_t zz_plan_workspace_bytes(const zz_plan_t* p) { return p ? p->ws.total : 0; }
 
 extern "C" zz_status_t zz_plan_upload(zz_plan_t* p, void* dev, size_t bytes, void* stream) {
+  ZZ_NVTX("zz_plan_upload");
   if (!p || !dev) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_upload: NULL argument");
   if (bytes < p->ws.total) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_upload: workspace too small");
   if (reinterpret_cast<uintptr_t>(dev) % 256)
@@ -363,7 +365,10 @@ extern "C" zz_status_t zz_plan_device_status(const zz_plan_t* p, int32_t* flags,
   if (e == cudaSuccess && clear) e = cudaMemsetAsync(st, 0, 4 * sizeof(int32_t), s);
   if (e != cudaSuccess)
     return zz::fail(ZZ_ERR_CUDA, std::string("zz_plan_device_status: ") + cudaGetErrorString(e));
-  if (*flags & 1)
+  if (*flags & zz::kStatusTimeout)
     return zz::fail(ZZ_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (pipeline stalled)");
+  if (*flags & zz::kStatusBadPage)
+    return zz::fail(ZZ_ERR_INVALID_ARG,
+                    "a page_table entry pointed outside the pool; its keys were read as zeros");
   return ZZ_OK;
 }

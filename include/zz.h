@@ -277,7 +277,7 @@ zz_status_t zz_ipc_close(void* base);
  * Errors: ZZ_ERR_INVALID_ARG when h_q % h_kv != 0 (message names "multiple of
  * num_kv_heads"), null or misaligned pointers, rank range outside [0,c);
  * ZZ_ERR_UNSUPPORTED for d not in {64,128}, or for bf16 a page_size that is
- * neither 16, 32, 64 nor a multiple of 128.
+ * neither 8, 16, 32, 64 nor a multiple of 128.
  * bf16 runs the tcgen05/TMEM/TMA kernel (fp32 accumulate and softmax); fp32
  * runs a CUDA-core kernel in full fp32.
  */

@@ -257,7 +257,7 @@ def rerange_push_kv(plan: Plan, rank: int, k_local, v_local, k_pools, v_pools, o
     tensor on this GPU or an int address (a peer pool mapped with ``PeerBuffer``).
     """
     n = len(k_pools)
-    if v_pools is not None and len(v_pools) != n or len(out_cache_locs) != n:
+    if (v_pools is not None and len(v_pools) != n) or len(out_cache_locs) != n:
         raise ValueError("k_pools, v_pools and out_cache_locs must have one entry per destination")
     kp = (_P * n)(*[_addr(x) for x in k_pools])
     vp = (_P * n)(*[_addr(x) for x in v_pools]) if v_pools is not None else None

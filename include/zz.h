@@ -60,7 +60,8 @@ typedef enum {
   ZZ_FIELD_Q_LEN_NEXT = 11,        /* [bs]      per rank (actual_seq_q_next)                   */
   ZZ_FIELD_CU_SEQLENS_Q_PREV = 12, /* [bs+1]    per rank, local exclusive prefix sums          */
   ZZ_FIELD_CU_SEQLENS_Q_NEXT = 13, /* [bs+1]    per rank                                       */
-  ZZ_FIELD_SRC_ROW = 14            /* [T]       natural token -> row of the [c*M] layout       */
+  ZZ_FIELD_SRC_ROW = 14,           /* [T]       natural token -> row of the [c*M] layout       */
+  ZZ_FIELD_RANK_TOK = 15           /* [c*M]     row of the [c*M] layout -> natural token, -1 pad */
 } zz_field_t;
 
 typedef struct {

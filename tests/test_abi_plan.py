@@ -53,6 +53,9 @@ def test_planner_matches_oracle_bit_exact(seed):
         ranked = R.ranked_layout(ids + 1, ref)          # 0 marks padding
         src_row = np.array(plan.get("src_row"))
         assert (ranked[src_row] == ids + 1).all()
+        # ranked row -> natural token (the push form's table) is the same layout, -1 on padding
+        rank_tok = np.array(plan.get("rank_tok"))
+        assert (rank_tok + 1 == ranked).all()
         for r in range(c):
             info = plan.info(r)
             assert info.total_q_prev == ref.total_q_prev[r]

@@ -39,7 +39,7 @@ FIELDS = {
     "extend_lens": 0, "prefix": 1, "split_list": 2, "zigzag_index": 3, "cp_reverse_index": 4,
     "reverse_split_len": 5, "per_rank_actual_token": 6, "max_rank_len": 7, "kv_len_prev": 8,
     "kv_len_next": 9, "q_len_prev": 10, "q_len_next": 11, "cu_seqlens_q_prev": 12,
-    "cu_seqlens_q_next": 13, "src_row": 14,
+    "cu_seqlens_q_next": 13, "src_row": 14, "rank_tok": 15,
 }
 PER_RANK_FIELDS = {"zigzag_index", "kv_len_prev", "kv_len_next", "q_len_prev", "q_len_next",
                    "cu_seqlens_q_prev", "cu_seqlens_q_next"}

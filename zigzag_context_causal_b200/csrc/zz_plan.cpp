@@ -312,6 +312,7 @@ extern "C" zz_status_t zz_plan_get(const zz_plan_t* p, int rank, zz_field_t fiel
     case ZZ_FIELD_CU_SEQLENS_Q_PREV: v = &p->cu_prev[rank]; break;
     case ZZ_FIELD_CU_SEQLENS_Q_NEXT: v = &p->cu_next[rank]; break;
     case ZZ_FIELD_SRC_ROW: v = &p->src_row; break;
+    case ZZ_FIELD_RANK_TOK: v = &p->rank_tok; break;
     default: return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_get: unknown field");
   }
   *count = int64_t(v->size());

@@ -35,9 +35,9 @@ typedef enum {
   ZZ_OK = 0,
   ZZ_ERR_INVALID_ARG = 1,      /* null/misaligned pointer, bad size, h_q % h_kv != 0, ... */
   ZZ_ERR_NOT_APPLICABLE = 2,   /* zigzag CP refuses the batch (zigzag.py, can_apply)      */
-  ZZ_ERR_UNSUPPORTED = 3,      /* valid request this build does not implement (d, dtype)  */
+  ZZ_ERR_UNSUPPORTED = 3,      /* valid request the library does not implement (d, dtype) */
   ZZ_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed                        */
-  ZZ_ERR_DEVICE_TIMEOUT = 5    /* a bounded device-side wait gave up (see zz_attn_status) */
+  ZZ_ERR_DEVICE_TIMEOUT = 5    /* a bounded device-side wait gave up (zz_plan_device_status) */
 } zz_status_t;
 
 typedef enum { ZZ_BF16 = 0, ZZ_FP32 = 1 } zz_dtype_t;

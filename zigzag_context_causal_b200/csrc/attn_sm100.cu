@@ -18,9 +18,10 @@
 //   warp  8    MMA issue (one thread) + TMEM allocation
 //   warp  9    TMA producer: Q once, then K/V stages (V_{j-1}, K_j) into a smem ring
 //   warps 10-11 idle
-// Launched at 168 registers a thread; the softmax warpgroups grow to 208 and
-// the third warpgroup shrinks to 88 (208 + 208 + 88 = 3 x 168 per SM
-// sub-partition), so a whole 128-column row of S stays in registers.
+// Launched at 168 registers a thread; the softmax warpgroups grow to 216 and
+// the third warpgroup shrinks to 72 (216 + 216 + 72 = 3 x 168 per SM
+// sub-partition), so a whole 128-column row of S stays in registers with no
+// spills.
 // TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [256+D,256+2D).
 // P (bf16, two per column) overwrites the first 64 columns of its S tile and
 // feeds the P.V MMA straight from TMEM.  The MMA order per K/V tile j is
@@ -56,7 +57,7 @@ namespace {
 using namespace zz::dev;
 
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
+constexpr uint32_t kRegsSoftmax = 216, kRegsOther = 72;
 constexpr int kWarpMma = 8;
 constexpr int kWarpLoad = 9;
 constexpr uint32_t kTmemCols = 512;

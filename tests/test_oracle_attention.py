@@ -159,3 +159,26 @@ def test_noncausal_union_equals_full_noncausal_attention():
     ref = np.concatenate([A.attention_half(q[starts[s]:starts[s + 1]], ks[s], vs[s], lens[s], 0.3,
                                            causal=False)[0] for s in range(2)])
     assert np.abs(o_tok - ref).max() < 1e-12
+
+
+def test_union_with_cached_prefix_equals_tail_of_full_attention():
+    """With a cached prefix, every extend token at position prefix + t sees keys
+    0 .. prefix + t: the ranks' halves, back in token order, equal the extend
+    rows of plain causal attention over the whole sequence (prefix included)."""
+    c, ext, pre, h_q, h_kv, d = 2, [23, 17], [5, 9], 4, 2, 8
+    full = [e + q for e, q in zip(ext, pre)]
+    p = P.build_metadata(c, sum(ext), seqs_len=full, extend_lens=ext)
+    assert p.prefix == pre
+    q_all = [_rand((n, h_q, d), 40 + s) for s, n in enumerate(full)]
+    k_all = [_rand((n, h_kv, d), 50 + s) for s, n in enumerate(full)]
+    v_all = [_rand((n, h_kv, d), 60 + s) for s, n in enumerate(full)]
+    q_ext = np.concatenate([q_all[s][pre[s]:] for s in range(2)])
+    scale = d ** -0.5
+    per_rank = [A.run_rank(p, r, R.shard(q_ext, p, r), k_all, v_all, scale) for r in range(c)]
+    o_tok = R.gather_kv(R.all_gather_padded([o for o, _ in per_rank], p), p)
+    l_tok = R.gather_kv(R.all_gather_padded([l for _, l in per_rank], p), p)
+    ref = [A.full_causal(q_all[s], k_all[s], v_all[s], scale) for s in range(2)]
+    ref_o = np.concatenate([ref[s][0][pre[s]:] for s in range(2)])
+    ref_l = np.concatenate([ref[s][1][pre[s]:] for s in range(2)])
+    assert np.abs(o_tok - ref_o).max() < 1e-12
+    assert np.abs(l_tok - ref_l).max() < 1e-12

@@ -70,3 +70,21 @@ def test_top_left_mask_is_caught_by_union_pin():
     rows = [i for i, t in enumerate(R.shard(np.arange(L), p, r)) if i >= p.total_q_prev[r]]
     tokens = R.shard(np.arange(L), p, r)[rows]
     assert np.abs(top_left - ref[tokens]).max() > 1e-3
+
+
+def test_dropped_prefix_in_kv_len_is_caught_by_prefix_union_pin():
+    """kv lengths that forget the cached prefix shift every row's key window."""
+    c, ext, pre, d = 2, [23, 17], [5, 9], 8
+    full = [e + q for e, q in zip(ext, pre)]
+    p = P.build_metadata(c, sum(ext), seqs_len=full, extend_lens=ext)
+    q_all = [_rand((n, 2, d), 70 + s) for s, n in enumerate(full)]
+    k_all = [_rand((n, 1, d), 80 + s) for s, n in enumerate(full)]
+    v_all = [_rand((n, 1, d), 90 + s) for s, n in enumerate(full)]
+    q_ext = np.concatenate([q_all[s][pre[s]:] for s in range(2)])
+    for kv in (p.kv_len_prev, p.kv_len_next):        # the planted mistake
+        for r in range(c):
+            kv[r] = [kv[r][s] - pre[s] for s in range(2)]
+    per_rank = [A.run_rank(p, r, R.shard(q_ext, p, r), k_all, v_all, 0.5)[0] for r in range(c)]
+    o_tok = R.gather_kv(R.all_gather_padded(per_rank, p), p)
+    ref = np.concatenate([A.full_causal(q_all[s], k_all[s], v_all[s], 0.5)[0][pre[s]:] for s in range(2)])
+    assert np.abs(o_tok - ref).max() > 1e-3

@@ -41,6 +41,7 @@ SMALL = [
     Case(2, [260, 300], 4, 2, 128, page_size=16, prefix=[100, 37]),   # cached prefix
     Case(2, [96], 2, 1, 128, page_size=16),                # every half shorter than one tile
     Case(2, [48], 2, 2, 64, dtype="fp32", page_size=16),   # fp32 paged
+    Case(3, [500, 129], 4, 4, 64, page_size=64),           # bf16 head_dim 64, MHA row-tile pairs
 ]
 
 

@@ -63,7 +63,8 @@ def test_bounded_wait_gives_up_and_context_stays_usable():
     Case(3, [700], 4, 4, 128, page_size=64, causal=False),              # row-pair mode
     Case(2, [260, 300], 4, 2, 128, page_size=16, prefix=[100, 37], causal=False),
     Case(2, [256], 4, 4, 64, dtype="fp32", page_size=256, scale=1.0, page_seed=None, causal=False),
-], ids=["gqa", "mha", "prefix", "fp32"])
+    Case(2, [333, 200], 4, 2, 64, page_size=32, causal=False),          # bf16 head_dim 64
+], ids=["gqa", "mha", "prefix", "fp32", "d64"])
 def test_noncausal_local_q_global_kv(case):
     _check_full(Run(case))
 

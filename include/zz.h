@@ -116,10 +116,11 @@ size_t zz_plan_workspace_bytes(const zz_plan_t* plan);
  * map, half descriptors, longest-first work lists) into `dev_workspace`
  * (caller-owned, >= zz_plan_workspace_bytes, 256-byte aligned) on `stream`,
  * and remember that address for later calls.  The plan must outlive the copy.
- * The source is the plan's own pageable host memory, so under CUDA's rules
- * for pageable copies the call returns only once `stream` has reached the copy
- * and the tables are staged: it is a once-per-batch call, made before the
- * kernels and outside stream capture, unlike the kernel entry points.
+ * The first upload of a plan lays its tables out in pinned host memory owned
+ * by the plan (cudaMallocHost, freed by zz_plan_destroy; make that first call
+ * outside stream capture).  Every upload is then one asynchronous copy from
+ * there, which neither waits for `stream` nor blocks the calling thread, and
+ * also clears the status word.
  */
 zz_status_t zz_plan_upload(zz_plan_t* plan, void* dev_workspace, size_t bytes, void* stream);
 

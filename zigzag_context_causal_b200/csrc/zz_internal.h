@@ -63,6 +63,7 @@ struct zz_plan {
   std::vector<int32_t> tile_rank_off, pair_rank_off;              // [c+1]
   zz::Workspace ws{};
   void* dev_ws = nullptr;
+  void* staging = nullptr;   // pinned host image of the workspace, made at the first upload
 };
 
 namespace zz {

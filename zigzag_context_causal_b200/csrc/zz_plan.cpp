@@ -269,7 +269,10 @@ extern "C" zz_status_t zz_plan_create(int cp_size, int bs, const int32_t* extend
   return ZZ_OK;
 }
 
-extern "C" void zz_plan_destroy(zz_plan_t* plan) { delete plan; }
+extern "C" void zz_plan_destroy(zz_plan_t* plan) {
+  if (plan && plan->staging) cudaFreeHost(plan->staging);
+  delete plan;
+}
 
 extern "C" zz_status_t zz_plan_info(const zz_plan_t* p, int rank, zz_plan_info_t* out) {
   if (!p || !out) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_info: NULL argument");
@@ -332,23 +335,31 @@ extern "C" zz_status_t zz_plan_upload(zz_plan_t* p, void* dev, size_t bytes, voi
   if (reinterpret_cast<uintptr_t>(dev) % 256)
     return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_upload: workspace must be 256-byte aligned");
   auto s = static_cast<cudaStream_t>(stream);
-  char* base = static_cast<char*>(dev);
-  struct Part { size_t off; const void* src; size_t n; } parts[] = {
-      {p->ws.src_row, p->src_row.data(), p->src_row.size() * sizeof(int32_t)},
-      {p->ws.rank_tok, p->rank_tok.data(), p->rank_tok.size() * sizeof(int32_t)},
-      {p->ws.halves, p->halves.data(), p->halves.size() * sizeof(zz::HalfDesc)},
-      {p->ws.tiles_all, p->tiles_all.data(), p->tiles_all.size() * sizeof(zz::WorkItem)},
-      {p->ws.tiles_rank, p->tiles_rank.data(), p->tiles_rank.size() * sizeof(zz::WorkItem)},
-      {p->ws.pairs_all, p->pairs_all.data(), p->pairs_all.size() * sizeof(zz::WorkItem)},
-      {p->ws.pairs_rank, p->pairs_rank.data(), p->pairs_rank.size() * sizeof(zz::WorkItem)},
-  };
-  for (auto& part : parts) {
-    if (!part.n) continue;
-    cudaError_t e = cudaMemcpyAsync(base + part.off, part.src, part.n, cudaMemcpyHostToDevice, s);
+  // The tables never change after zz_plan_create: lay them out once in pinned
+  // host memory exactly as in the workspace (status word zero), so that every
+  // upload is one asynchronous copy that neither waits for the stream nor
+  // blocks the calling thread.
+  if (!p->staging) {
+    void* h = nullptr;
+    cudaError_t e = cudaMallocHost(&h, p->ws.total);
     if (e != cudaSuccess)
-      return zz::fail(ZZ_ERR_CUDA, std::string("zz_plan_upload: ") + cudaGetErrorString(e));
+      return zz::fail(ZZ_ERR_CUDA, std::string("zz_plan_upload: pinned staging: ") + cudaGetErrorString(e));
+    char* img = static_cast<char*>(h);
+    std::memset(img, 0, p->ws.total);
+    struct Part { size_t off; const void* src; size_t n; } parts[] = {
+        {p->ws.src_row, p->src_row.data(), p->src_row.size() * sizeof(int32_t)},
+        {p->ws.rank_tok, p->rank_tok.data(), p->rank_tok.size() * sizeof(int32_t)},
+        {p->ws.halves, p->halves.data(), p->halves.size() * sizeof(zz::HalfDesc)},
+        {p->ws.tiles_all, p->tiles_all.data(), p->tiles_all.size() * sizeof(zz::WorkItem)},
+        {p->ws.tiles_rank, p->tiles_rank.data(), p->tiles_rank.size() * sizeof(zz::WorkItem)},
+        {p->ws.pairs_all, p->pairs_all.data(), p->pairs_all.size() * sizeof(zz::WorkItem)},
+        {p->ws.pairs_rank, p->pairs_rank.data(), p->pairs_rank.size() * sizeof(zz::WorkItem)},
+    };
+    for (auto& part : parts)
+      if (part.n) std::memcpy(img + part.off, part.src, part.n);
+    p->staging = h;
   }
-  cudaError_t e = cudaMemsetAsync(base + p->ws.status, 0, 4 * sizeof(int32_t), s);
+  cudaError_t e = cudaMemcpyAsync(dev, p->staging, p->ws.total, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess)
     return zz::fail(ZZ_ERR_CUDA, std::string("zz_plan_upload: ") + cudaGetErrorString(e));
   p->dev_ws = dev;

@@ -278,28 +278,28 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           __syncwarp();
         }
       }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bars->kv_full[slot], tma_bytes);
-        for (int which = 0; which < 2; ++which) {
-          const int tile_j = which ? t : t - 1;
-          if (tile_j < 0 || tile_j >= n_max) continue;
-          uint8_t* tile = stage + which * C::kTileBytes;
-          const void* tm = which ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
-          const int key0 = tile_j * 128;
-          for (int c = 0; c < chunks; ++c) {
-            const int kc = key0 + c * p.box_rows;
-            if (kc + p.box_rows > kv_end) continue;
-            // A page outside the pool is loaded from a coordinate past the pool's
-            // end (zero fill) and reported through the status word.
-            const int32_t page = __ldg(pt + kc / p.page_size);
-            const bool in_pool = uint32_t(page) < uint32_t(p.num_pages);
-            bad_page |= !in_pool;
-            const int32_t slot0 = (in_pool ? page : p.num_pages) * p.page_size + kc % p.page_size;
-            for (int b = 0; b < C::kBoxes; ++b)
-              tma_load_3d(tile + b * C::kBoxBytes + c * p.box_rows * 128, tm, &bars->kv_full[slot],
-                          b * 64, kv_head, slot0);
-          }
-        }
+      // Lane 0 posts the byte count first; then one lane per page chunk (up to
+      // 2 x 16 chunks for 8-token pages) reads its page-table entry and issues
+      // that chunk's boxes, so small pages cost one lookup latency per stage.
+      if (lane == 0) mbar_arrive_expect_tx(&bars->kv_full[slot], tma_bytes);
+      __syncwarp();
+      for (int u = lane; u < 2 * chunks; u += 32) {
+        const int which = u / chunks, c = u - which * chunks;
+        const int tile_j = which ? t : t - 1;
+        if (tile_j < 0 || tile_j >= n_max) continue;
+        const int kc = tile_j * 128 + c * p.box_rows;
+        if (kc + p.box_rows > kv_end) continue;
+        uint8_t* tile = stage + which * C::kTileBytes;
+        const void* tm = which ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
+        // A page outside the pool is loaded from a coordinate past the pool's
+        // end (zero fill) and reported through the status word.
+        const int32_t page = __ldg(pt + kc / p.page_size);
+        const bool in_pool = uint32_t(page) < uint32_t(p.num_pages);
+        bad_page |= !in_pool;
+        const int32_t slot0 = (in_pool ? page : p.num_pages) * p.page_size + kc % p.page_size;
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_3d(tile + b * C::kBoxBytes + c * p.box_rows * 128, tm, &bars->kv_full[slot],
+                      b * 64, kv_head, slot0);
       }
       __syncwarp();
     }

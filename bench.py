@@ -111,6 +111,90 @@ def push_all_local(zz, plan, r0: int, r_per: int, M: int, k_local, v_local, dsts
                            [loc] * len(dsts[0]), num_slots)
 
 
+def kv_exchange(world: int, push: bool, fence, push_fn, gather_fn, rerange_fn) -> None:
+    """The exchange step of one pass: K/V of every rank into this rank's pool.
+
+    All-gather form: all-gather the shards (N > 1), then the rerange kernel.
+    Push form: every rank's kernel writes straight into every rank's pool, so
+    the pools are shared state and need a fence on both sides of the push:
+      * before it (write after read): every rank's previous attention has
+        finished reading its pool before anyone overwrites it;
+      * after it (read after write): every rank's rows have landed before any
+        attention reads them.
+    ``fence`` is a stream-ordered collective (a one-element all-reduce): the
+    same step on every rank, in the same order."""
+    if push:
+        if world > 1:
+            fence()
+        push_fn()
+        if world > 1:
+            fence()
+    else:
+        if world > 1:
+            gather_fn()
+        rerange_fn()
+
+
+class RankFailure(RuntimeError):
+    """A peer rank did not reach a step within the heartbeat timeout."""
+
+
+def heartbeat(store, tag: str, rank: int, world: int, timeout_s: float) -> None:
+    """Host-side liveness check between steps: every rank posts ``tag`` in the
+    process group's store and waits, at most ``timeout_s``, for every other
+    rank's post.  A rank that left (exited, crashed, or stopped between steps)
+    is reported by name before this rank launches the step's collectives,
+    instead of being found by a collective that waits for it."""
+    from datetime import timedelta
+    store.set(f"zz_hb/{tag}/{rank}", "1")
+    keys = [f"zz_hb/{tag}/{r}" for r in range(world) if r != rank]
+    try:
+        store.wait(keys, timedelta(seconds=timeout_s))
+    except Exception as e:  # the store raises on timeout (the type varies by store)
+        missing = []
+        for r in range(world):
+            if r == rank:
+                continue
+            try:
+                present = store.check([f"zz_hb/{tag}/{r}"])
+            except Exception:
+                present = False
+            if not present:
+                missing.append(r)
+        raise RankFailure(f"rank {rank}: ranks {missing} did not reach {tag} within {timeout_s:.1f} s") from e
+
+
+def gather_buffers(dist, torch, dev, shape, dtype, world: int):
+    """Targets of the K and V all-gathers.
+
+    On NCCL they come from NCCL's own allocator and are registered with the
+    process group, the way the zigzag page allocates the gathered K/V under a
+    symmetric-memory context before its all-gather (``_all_gather_reorganized``),
+    so NCCL can write peers' rows straight into them.  The rerange kernel then
+    reads them in place.  Returns (k, v, registration); registration is passed
+    to ``release_gather_buffers`` before the process group is destroyed."""
+    if world > 1 and dist.get_backend() == "nccl":
+        try:
+            backend = dist.group.WORLD._get_backend(dev)
+            pool = torch.cuda.MemPool(backend.mem_allocator)
+            with torch.cuda.use_mem_pool(pool):
+                k = torch.zeros(shape, dtype=dtype, device=dev)
+                v = torch.zeros(shape, dtype=dtype, device=dev)
+            backend.register_mem_pool(pool)
+            return k, v, {"backend": backend, "pool": pool, "kind": "nccl-registered"}
+        except Exception as e:  # registration is an optimisation of the same collective
+            note = f"plain (NCCL registration unavailable: {type(e).__name__}: {e})"
+            return (torch.zeros(shape, dtype=dtype, device=dev), torch.zeros(shape, dtype=dtype, device=dev),
+                    {"kind": note[:200]})
+    return (torch.zeros(shape, dtype=dtype, device=dev), torch.zeros(shape, dtype=dtype, device=dev),
+            {"kind": "plain"})
+
+
+def release_gather_buffers(reg) -> None:
+    if reg and "pool" in reg:
+        reg["backend"].deregister_mem_pool(reg["pool"])
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -293,8 +377,7 @@ def main_gpu(args):
     q_all = torch.zeros(cp * M, h_q, d, dtype=torch.bfloat16, device=dev)
     zz.shard_rows(plan, q_nat, q_all)
     q_mine = q_all[r0 * M:(r0 + r_per) * M].contiguous()
-    k_g = torch.zeros(cp * M, h_kv, d, dtype=torch.bfloat16, device=dev)
-    v_g = torch.zeros_like(k_g)
+    k_g, v_g, gather_reg = gather_buffers(dist, torch, dev, (cp * M, h_kv, d), torch.bfloat16, world)
     zz.shard_rows(plan, k_nat, k_g)
     zz.shard_rows(plan, v_nat, v_g)
     k_local = k_g[r0 * M:(r0 + r_per) * M].contiguous()
@@ -321,20 +404,22 @@ def main_gpu(args):
         else:
             dsts = [[k_pool], [v_pool]]
 
+    store = dist.distributed_c10d._get_default_store() if world > 1 else None
+    fence = (lambda: dist.all_reduce(fence_t)) if push and world > 1 else None
+    step_no = [0]
+
     def step(record: bool):
         # S1 plan tables, S3 (multi-GPU only) all-gather, S4 rerange, S5 attention
+        if world > 1:   # every peer is still here before this step's collectives
+            heartbeat(store, f"step{step_no[0]}", rank, world, args.heartbeat_s)
+        step_no[0] += 1
         plan.upload(ws)
-        if world > 1 and not push:
-            all_gather_rows(dist, k_g, k_local)
-            all_gather_rows(dist, v_g, v_local)
         e0, e1, e2 = ev(), ev(), ev()
         e0.record(stream)
-        if push:
-            push_all_local(zz, plan, r0, r_per, M, k_local, v_local, dsts, loc, pool.num_slots)
-            if world > 1:   # stream-ordered: every rank's pushes done before anyone's attention
-                dist.all_reduce(fence_t)
-        else:
-            zz.rerange_kv_to_pool(plan, k_g, v_g, k_pool, v_pool, loc)
+        kv_exchange(world, push, fence,
+                    lambda: push_all_local(zz, plan, r0, r_per, M, k_local, v_local, dsts, loc, pool.num_slots),
+                    lambda: (all_gather_rows(dist, k_g, k_local), all_gather_rows(dist, v_g, v_local)),
+                    lambda: zz.rerange_kv_to_pool(plan, k_g, v_g, k_pool, v_pool, loc))
         e1.record(stream)
         zz.attn_prefill(plan, q_mine, k_pool, v_pool, page_table, ps, out, softmax_scale=scale,
                         rank_begin=r0, rank_count=r_per)
@@ -418,19 +503,17 @@ def main_gpu(args):
             if used[bi]:
                 stream.wait_event(ev_d2h[bi])        # step i-2's output has been read back
             plan.upload(ws)
-            if push:
-                push_all_local(zz, plan, r0, r_per, M, k_ds[bi], v_ds[bi], dsts, loc, pool.num_slots)
-                if world > 1:
-                    dist.all_reduce(fence_t)
-                kg_i, vg_i = None, None
-            elif world > 1:
-                all_gather_rows(dist, k_g, k_ds[bi])
-                all_gather_rows(dist, v_g, v_ds[bi])
+            if world > 1:
+                heartbeat(store, f"e2e{i}", rank, world, args.heartbeat_s)
+            if push or world > 1:
                 kg_i, vg_i = k_g, v_g
-            else:
+            else:   # one GPU: the copied-in shard is the whole gathered buffer
                 kg_i, vg_i = k_ds[bi], v_ds[bi]
-            if kg_i is not None:
-                zz.rerange_kv_to_pool(plan, kg_i, vg_i, k_pool, v_pool, loc)
+            kv_exchange(world, push, fence,
+                        lambda: push_all_local(zz, plan, r0, r_per, M, k_ds[bi], v_ds[bi], dsts, loc,
+                                               pool.num_slots),
+                        lambda: (all_gather_rows(dist, k_g, k_ds[bi]), all_gather_rows(dist, v_g, v_ds[bi])),
+                        lambda: zz.rerange_kv_to_pool(plan, kg_i, vg_i, k_pool, v_pool, loc))
             for k in range(r_per):
                 stream.wait_event(ev_q[bi][k])
                 zz.attn_prefill(plan, q_ds[bi][k * M:(k + 1) * M], k_pool, v_pool, page_table, ps,
@@ -484,10 +567,18 @@ def main_gpu(args):
         for m in mapped:
             m.close()
         dist.barrier()
+    release_gather_buffers(gather_reg)
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return 0
+
+    # ---- every configuration's shape, one GPU (rank 0), after the main step's buffers are gone
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        del q_mine, out, k_local, v_local, k_g, v_g, k_pool, v_pool
+        torch.cuda.empty_cache()
+        per_config = per_config_attention(torch, zz, synth, dev)
 
     peaks, peaks_src = load_peaks()
     peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
@@ -515,14 +606,16 @@ def main_gpu(args):
         "config": {"workload": desc, "cp_size": cp, "seq_lens": lens if len(lens) <= 8 else len(lens),
                    "h_q": h_q, "h_kv": h_kv, "head_dim": d, "page_size": ps,
                    "parallelism": f"zigzag-cp{cp} (virtual ranks {r_per}/GPU)",
-                   "kv_exchange": args.kv_exchange,
+                   "kv_exchange": args.kv_exchange, "gather_buffer": gather_reg["kind"],
                    "l2": "no flush: Q 2 GiB, gathered K/V 2x256 MiB and pool exceed the 126 MB L2"
                    if args.workload == "long" else "inputs sized per workload"},
         "attn_kernel_ms": attn_kernel_ms, "attn_tflops": attn_tflops,
         "attn_frac_of_bf16_sustained": attn_tflops / peak_sus,
         "attn_frac_of_bf16_burst": attn_tflops / peak_burst,
         "rerange_kernel_ms": rr_kernel_ms, "rerange_gbs": rr_bytes / (rr_kernel_ms * 1e-3) / 1e9,
+        "attn_per_clock": per_clock(attn_tflops, clocks),
         "rerange_standalone": rerange_sweep,
+        "per_config": per_config,
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_sm100", "achieved": attn_tflops,
                      "peak": peak_sus, "unit": "TFLOP/s", "frac": attn_tflops / peak_sus,
                      "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel runs inside a long step)",
@@ -537,6 +630,111 @@ def main_gpu(args):
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+# Dense bf16 tensor-core work of one SM per clock on B200 (one 128x128x16 MMA,
+# 524288 FLOPs, every 64 cycles), and the SM count.
+TENSOR_FLOP_PER_SM_CYCLE = 8192
+B200_SMS = 148
+
+
+def per_clock(tflops: float, clocks: dict):
+    """Tensor-core work per SM clock, as a fraction of the dense bf16 rate per
+    clock: the figure that power-capped clocks do not move."""
+    mhz = clocks.get("sm_mhz") if clocks else None
+    if not mhz:
+        return None
+    flop_per_cycle = tflops * 1e12 / (mhz * 1e6) / B200_SMS
+    return {"sm_mhz": mhz, "flop_per_sm_cycle": flop_per_cycle,
+            "frac_of_dense_bf16_per_cycle": flop_per_cycle / TENSOR_FLOP_PER_SM_CYCLE}
+
+
+# Every configuration's shape (causal attention).  name: (cp, lens, h_q, h_kv, d,
+# page_size, dtype, value_scale, page_seed)
+PER_CONFIG = [
+    ("1: c=2 L=256 4/4 D=64 fp32 unpaged", 2, [256], 4, 4, 64, 256, "fp32", 1.0, None),
+    ("2: c=4 L=4096 32/4 D=128 bf16 page 16", 4, [4096], 32, 4, 128, 16, "bf16", 0.5, 1),
+    ("3: c=4 varlen x8 U[1000,8192] 32/4 D=128 bf16 page 16", 4, "varlen", 32, 4, 128, 16, "bf16", 0.5, 1),
+    ("4: c=8 L=131072 64/8 D=128 bf16 page 64", 8, [131072], 64, 8, 128, 64, "bf16", 0.5, 1),
+] + [(f"5: c={cp} L=32768 {hq}/{hkv} D=128 bf16 page 16", cp, [32768], hq, hkv, 128, 16, "bf16", 0.5, 1)
+     for hq, hkv in ((32, 32), (32, 8), (32, 1)) for cp in (2, 4, 8)]
+
+
+def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 512):
+    """Attention (and rerange) kernel time on every configuration's shape.
+
+    Per configuration: seeded inputs, plan, shard, rerange into the paged pool,
+    then ``reps`` timed launches of each kernel, each launch preceded by a write
+    of ``flush_mb`` MB (so every launch starts with a cold L2), each timed alone
+    with CUDA events on the launching stream; the median is reported.  FLOPs
+    are the exact causal pairs x 4 * D * H_q; rerange bytes are K and V, read
+    once and written once.  The long-context shape is the step above; it is
+    timed here again in the same short-launch way for comparison."""
+    peaks, src = load_peaks()
+    burst = float(peaks.get("bf16_tflops"))
+    sus = float(peaks.get("bf16_tflops_sustained", burst))
+    hbm = float(peaks["hbm_gbs"])
+    flush = torch.empty(flush_mb << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    out_rows = []
+    for name, cp, spec, h_q, h_kv, d, ps, dtype, vscale, pseed in PER_CONFIG:
+        lens = _lens(spec)
+        T = sum(lens)
+        plan = zz.Plan(cp, extend_lens=lens)
+        plan.upload()
+        M = plan.M
+        q_nat, k_nat, v_nat = synth.qkv(T, h_q, h_kv, d, seed=0, scale=vscale, dtype=dtype, device=str(dev))
+        tdt = q_nat.dtype
+        q = torch.zeros(cp * M, h_q, d, dtype=tdt, device=dev)
+        kg = torch.zeros(cp * M, h_kv, d, dtype=tdt, device=dev)
+        vg = torch.zeros_like(kg)
+        zz.shard_rows(plan, q_nat, q)
+        zz.shard_rows(plan, k_nat, kg)
+        zz.shard_rows(plan, v_nat, vg)
+        del q_nat, k_nat, v_nat
+        pool = synth.paged_pool(lens, ps, seed=pseed)
+        page_table = torch.from_numpy(pool.page_table).to(dev)
+        loc = torch.from_numpy(pool.out_cache_loc).to(dev)
+        kp = torch.zeros(pool.num_slots, h_kv, d, dtype=tdt, device=dev)
+        vp = torch.zeros_like(kp)
+        out = torch.empty_like(q)
+        scale = 1.0 / math.sqrt(d)
+        flops = 4 * d * h_q * plan.causal_pairs
+        rr_bytes = 2 * 2 * T * h_kv * d * q.element_size()
+
+        def timed(fn):
+            ts = []
+            for i in range(reps + 1):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                if i:                    # the first launch warms the code path
+                    ts.append(a.elapsed_time(b))
+            return statistics.median(ts)
+
+        rr_ms = timed(lambda: zz.rerange_kv_to_pool(plan, kg, vg, kp, vp, loc))
+        at_ms = timed(lambda: zz.attn_prefill(plan, q, kp, vp, page_table, ps, out, softmax_scale=scale))
+        status = plan.device_status(clear=True)
+        tf = flops / (at_ms * 1e-3) / 1e12
+        row = {"config": name, "attn_ms": at_ms, "attn_tflops": tf, "flops": flops,
+               "rerange_us": rr_ms * 1e3, "rerange_gbs": rr_bytes / (rr_ms * 1e-3) / 1e9,
+               "rerange_frac_of_hbm": rr_bytes / (rr_ms * 1e-3) / 1e9 / hbm, "device_status": status}
+        if dtype == "bf16":
+            row["attn_frac_of_bf16_burst"] = tf / burst
+            row["attn_frac_of_bf16_sustained"] = tf / sus
+        else:
+            row["attn_kernel"] = "fp32 CUDA-core kernel (no tensor-core peak applies)"
+        out_rows.append(row)
+        del q, kg, vg, kp, vp, out, page_table, loc, plan
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return {"rows": out_rows, "peak_source": f"{src} (burst: launches of at most ~0.25 s, timed alone)",
+            "method": f"median of {reps} launches per kernel, each after a {flush_mb} MB L2 flush, "
+                      "CUDA events on the launching stream"}
 
 
 KERNEL_SOURCES = {
@@ -717,6 +915,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rerange-sweep", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the attention timing on every configuration's shape")
+    ap.add_argument("--heartbeat-s", type=float, default=120.0,
+                    help="N > 1: how long a rank waits for its peers at each step before it reports them gone")
     ap.add_argument("--kv-exchange", default="allgather", choices=["allgather", "push"],
                     help="allgather: NCCL all-gather then the rerange kernel; push: every rank's "
                          "kernel writes its rows straight into every rank's pool (IPC-mapped)")

@@ -131,7 +131,11 @@ zz_status_t zz_plan_upload(zz_plan_t* plan, void* dev_workspace, size_t bytes, v
  * points outside the pool (those keys were read as zeros).  Synchronises
  * `stream` (a diagnostic, not a hot-path call).  Returns ZZ_ERR_DEVICE_TIMEOUT
  * when bit 0 is set, else ZZ_ERR_INVALID_ARG when bit 2 is set, else ZZ_OK.
- * zz_plan_upload clears the word.
+ * zz_plan_upload clears the word.  When the plan's last zz_attn_prefill_noalloc
+ * call ran on the current device, the status word of the library's static
+ * array is read (and cleared) too, and *flags is the OR of both words.
+ * ZZ_ERR_INVALID_ARG if the plan was neither uploaded nor used by
+ * zz_attn_prefill_noalloc.
  */
 zz_status_t zz_plan_device_status(const zz_plan_t* plan, int32_t* flags, int clear, void* stream);
 
@@ -226,10 +230,16 @@ enum { ZZ_MAX_PUSH_DST = 16 };
  *     readable by the calling GPU (one map may serve every destination).
  * v_local and v_pools may both be NULL (one tensor).  1 <= n_dst <=
  * ZZ_MAX_PUSH_DST.  Slots outside [0, num_slots) are skipped.  The call only
- * enqueues the kernel: before any rank reads its pool, every rank's push into
- * it must have completed (e.g. a stream-ordered collective or a host barrier
- * after each rank's kernel).  Bit-exact copy; row h_kv*d*sizeof(dtype) a
- * multiple of 16 bytes and every pointer 16-byte aligned.
+ * enqueues the kernel; the caller orders it against the other ranks both ways:
+ *   - read after write: before any rank reads its pool, every rank's push into
+ *     it must have completed (e.g. a stream-ordered collective after each
+ *     rank's push kernel);
+ *   - write after read: before a rank pushes new rows into the pools, every
+ *     rank must have finished reading the previous contents of its own pool
+ *     (its attention), e.g. a stream-ordered collective after each rank's
+ *     attention, or pools used in alternation (double buffering).
+ * Bit-exact copy; row h_kv*d*sizeof(dtype) a multiple of 16 bytes and every
+ * pointer 16-byte aligned.
  * The pages gather first and rerange after; the push form is this library's
  * own, and on one GPU it equals zz_rerange_kv_to_pool run per rank.
  */
@@ -323,26 +333,35 @@ zz_status_t zz_attn_prefill_ex(const zz_plan_t* plan, int rank_begin, int rank_c
                                float softmax_scale, zz_dtype_t dtype, uint32_t flags, void* stream);
 
 /*
- * zz_attn_prefill without a workspace (bf16 only).  The zigzag pages have no
- * counterpart to this call; it exists for callers that cannot hand the library
- * device memory they allocated themselves: code that must not call
- * cudaMalloc (for example while a CUDA graph is being captured, or inside a
- * runtime whose memory is owned by its own arena allocator), and callers that
- * want no device allocation tied to the life of a plan.
+ * zz_attn_prefill without a workspace (bf16, causal).  The zigzag pages have
+ * no counterpart to this call.  It is for callers that cannot hand the library
+ * device memory of their own: a host runtime whose device memory all belongs
+ * to its own arena and that gives plug-ins no allocation call, or a process
+ * that must keep its device footprint fixed after start-up and so may not
+ * call cudaMalloc (or an allocator that ends in it) per request.
  *
- * Same arguments and results as zz_attn_prefill.  zz_plan_upload is not
- * needed: the half table, the work list and the status word are copied on
- * `stream` into a file-scope __device__ array of 1 MiB that lives inside the
- * library (every GPU that loads libzz keeps it until the process exits).  The
- * call itself allocates nothing and calls no cudaMalloc or cudaFree.
+ * Same arguments and results as zz_attn_prefill (bit for bit: the same kernel
+ * reads the same tables).  zz_plan_upload is not needed.  The half table, the
+ * work list and a status word live in a file-scope __device__ array of 1 MiB
+ * inside the library instead of a workspace; every GPU that loads libzz holds
+ * that array until the process exits.  The call allocates nothing, host or
+ * device: it calls no cudaMalloc, cudaMallocHost or cudaFree.  The tables
+ * travel to the array as kernel parameters of small copy launches (1 per
+ * 32 640 bytes of tables) enqueued on `stream` before the attention launch,
+ * so the call neither waits for the stream nor blocks the calling thread.
  *   - Plans whose tables need more than 1 MiB (half table plus work list,
- *     about 130 000 work items) are rejected with ZZ_ERR_INVALID_ARG before
- *     anything is enqueued.
+ *     about 130 000 work items) are rejected with ZZ_ERR_INVALID_ARG, like
+ *     every other invalid call, before anything is enqueued.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
- *   - All calls share the one array and the last call's tables stay in it; the
- *     status word is cleared by every call.  Calls whose work overlaps on the
- *     GPU (other streams, other host threads) race on the array: serialise them.
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - All calls share the one array and the last call's tables stay in it.
+ *     Each call clears the status word before its attention launch.  Calls
+ *     whose work overlaps on the GPU (other streams, other host threads) race
+ *     on the array and must be serialised by the caller.
+ *   - Device-side errors (a bounded wait that gave up, a page_table entry
+ *     outside the pool) set the array's status word; zz_plan_device_status on
+ *     the same plan, with the same device current, reads and clears it.
  */
 zz_status_t zz_attn_prefill_noalloc(const zz_plan_t* plan, int rank_begin, int rank_count,
                                     const void* q, const void* k_pool, const void* v_pool,

@@ -123,24 +123,55 @@ class Run:
                         out.append((r, base + cu[s] + j, h, s, j))
         return out
 
-    def expected_rows(self, samples):
-        """Oracle o, lse for sampled rows (computed one row block at a time)."""
+    def tile_rows(self, rng_seed: int = 0, tile: int = 128):
+        """One row from EVERY ``tile``-row query tile of every half (at an offset
+        that changes from tile to tile, so both 128-row sub-tiles of a CTA, every
+        work item and every position inside a tile get exercised), plus the
+        first and last row of each half."""
         p = self.ref_plan
-        q_nat = self.q
-        res = []
+        rng = np.random.default_rng(rng_seed)
+        out = []
+        for r in range(p.cp_size):
+            for h, (cu, base) in enumerate(((p.cu_seqlens_q_prev[r], 0),
+                                            (p.cu_seqlens_q_next[r], p.total_q_prev[r]))):
+                for s in range(p.bs):
+                    lq = cu[s + 1] - cu[s]
+                    rows = {0, lq - 1}
+                    for t0 in range(0, lq, tile):
+                        rows.add(t0 + int(rng.integers(0, min(tile, lq - t0))))
+                    for j in sorted(rows):
+                        out.append((r, base + cu[s] + j, h, s, j))
+        return out
+
+    def expected_rows(self, samples):
+        """Oracle o, lse for sampled rows, one oracle call per (rank, half,
+        sequence) so that each half's keys are read once."""
+        p = self.ref_plan
         ks = [k.double().cpu().numpy() for k in self.k_seqs]
         vs = [v.double().cpu().numpy() for v in self.v_seqs]
-        tok_of = {}
         starts = np.cumsum([0] + self.case.lens)
-        for (r, lrow, h, s, j) in samples:
+        groups = {}
+        for i, (r, lrow, h, s, j) in enumerate(samples):
+            groups.setdefault((r, h, s), []).append((i, j))
+        res = [None] * len(samples)
+        for (r, h, s), members in groups.items():
             kv_len = (p.kv_len_prev if h == 0 else p.kv_len_next)[r][s]
             lq = (p.q_len_prev if h == 0 else p.q_len_next)[r][s]
             blk = r if h == 0 else 2 * p.cp_size - 1 - r
-            tok = starts[s] + sum(p.blocks[s][:blk]) + j            # natural token of this row
-            qrow = q_nat[tok:tok + 1].double().cpu().numpy()
-            o, l = OA.attention_rows(qrow, [j], ks[s], vs[s], kv_len, lq, self.softmax_scale)
-            res.append((o[0], l[0]))
+            first_tok = starts[s] + sum(p.blocks[s][:blk])             # natural token of row 0
+            js = np.array([j for _, j in members])
+            idx = torch.from_numpy(first_tok + js).to(self.q.device)
+            qrows = self.q[idx].double().cpu().numpy()
+            o, l = OA.attention_rows(qrows, js, ks[s], vs[s], kv_len, lq, self.softmax_scale)
+            for n, (i, _) in enumerate(members):
+                res[i] = (o[n], l[n])
         return res
+
+    def padding_rows(self):
+        """Rows of the [c*M] layout that belong to no half (never to be written)."""
+        p = self.ref_plan
+        return np.concatenate([np.arange(r * p.M + n, (r + 1) * p.M)
+                               for r, n in enumerate(p.per_rank_actual_token)]).astype(np.int64)
 
 
 def assert_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str = ""):

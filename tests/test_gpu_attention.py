@@ -1,8 +1,11 @@
 """Attention parity with the fp64 oracle (GPU), through the C ABI.
 
 Small cases are compared on every valid output row; the full-size
-configurations on sampled rows (first, last and random rows of every half of
-every rank).  Tolerances: bf16 max-abs 2e-2 and mean-abs 2e-3, fp32 max-abs 1e-4.
+configurations on one row of EVERY 128-row query tile of every half of every
+rank (at an offset that varies from tile to tile) plus each half's first and
+last row, so every work item and both query sub-tiles of each CTA are checked.
+Rows of the [c*M] layout that belong to no half must stay unwritten (NaN).
+Tolerances: bf16 max-abs 2e-2 and mean-abs 2e-3, fp32 max-abs 1e-4.
 """
 import numpy as np
 import pytest
@@ -27,6 +30,14 @@ def _check_full(run: Run):
         assert np.isfinite(got).all()
         assert_close(got, o_ref, run.case.dtype, f"rank {r} out")
         assert np.abs(lse[r * p.M: r * p.M + n] - l_ref).max() < 2e-3, f"rank {r} lse"
+    _check_padding_untouched(run)
+
+
+def _check_padding_untouched(run: Run):
+    pad = torch.from_numpy(run.padding_rows()).to(run.out.device)
+    if pad.numel():
+        assert torch.isnan(run.out.index_select(0, pad).float()).all(), "a padding row was written"
+        assert torch.isnan(run.lse.index_select(0, pad)).all(), "a padding row's lse was written"
 
 
 SMALL = [
@@ -82,30 +93,32 @@ def test_union_in_token_order_equals_unsharded_attention():
     assert_close(o_tok, ref, "bf16", "union")
 
 
-def _check_sampled(run: Run, per_half: int):
+def _check_sampled(run: Run, per_half: int | None = None):
+    """per_half=None: one row of every query tile; else first/last + random rows."""
     run.attend()
-    samples = run.sampled_rows(per_half)
+    samples = run.tile_rows() if per_half is None else run.sampled_rows(per_half)
     want = run.expected_rows(samples)
-    out = run.out
-    lse = run.lse
     p = run.ref_plan
-    got = np.stack([out[r * p.M + lrow].float().cpu().numpy() for (r, lrow, *_rest) in samples])
+    idx = torch.tensor([r * p.M + lrow for (r, lrow, *_rest) in samples], device=run.out.device)
+    got = run.out.index_select(0, idx).float().cpu().numpy()
     ref = np.stack([w[0] for w in want])
     assert np.isfinite(got).all()
-    assert_close(got, ref, "bf16", "sampled rows")
-    gl = np.stack([lse[r * p.M + lrow].cpu().numpy() for (r, lrow, *_rest) in samples])
+    assert_close(got, ref, "bf16", f"{len(samples)} sampled rows")
+    gl = run.lse.index_select(0, idx).cpu().numpy()
     assert np.abs(gl - np.stack([w[1] for w in want])).max() < 2e-3
+    _check_padding_untouched(run)
 
 
-def test_varlen_batch_c4_sampled_rows():
+def test_varlen_batch_c4_every_tile():
     lens = synth.varlen_lengths(8, 1000, 8192, seed=0)
-    _check_sampled(Run(Case(4, lens, 32, 4, 128, page_size=16)), per_half=6)
+    _check_sampled(Run(Case(4, lens, 32, 4, 128, page_size=16)))
 
 
-@pytest.mark.parametrize("h_q,h_kv,cp", [(32, 32, 2), (32, 8, 4), (32, 1, 8)])
-def test_L32768_head_ratio_sweep_sampled_rows(h_q, h_kv, cp):
-    _check_sampled(Run(Case(cp, [32768], h_q, h_kv, 128, page_size=16)), per_half=3)
+@pytest.mark.parametrize("cp", [2, 4, 8])
+@pytest.mark.parametrize("h_q,h_kv", [(32, 32), (32, 8), (32, 1)], ids=["mha", "gqa4", "mqa"])
+def test_L32768_head_ratio_sweep_every_tile(h_q, h_kv, cp):
+    _check_sampled(Run(Case(cp, [32768], h_q, h_kv, 128, page_size=16)))
 
 
-def test_long_context_c8_L131072_sampled_rows():
-    _check_sampled(Run(Case(8, [131072], 64, 8, 128, page_size=64)), per_half=2)
+def test_long_context_c8_L131072_every_tile():
+    _check_sampled(Run(Case(8, [131072], 64, 8, 128, page_size=64)))

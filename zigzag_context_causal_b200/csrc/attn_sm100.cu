@@ -36,6 +36,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <algorithm>
+#include <cstring>
 #include <mutex>
 #include <string>
 
@@ -544,13 +546,30 @@ zz_status_t encode_3d(CUtensorMap* m, const void* base, int d, int heads, int64_
 // Items per scheduling chunk: enough that one K/V head's blocks of a chunk
 // fill every SM once (one resident CTA per SM).
 int chunk_items_for(int groups_per_kv) {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+  return std::max(1, (device_sm_count() + groups_per_kv - 1) / groups_per_kv);
+}
+
+// The kernel needs more than 48 KB of dynamic shared memory, which must be
+// opted into once per function and device (the attribute belongs to the
+// device's context); remembered per device ordinal, guarded for host threads.
+constexpr int kMaxDevices = 256;
+std::mutex g_attr_mu;
+bool g_attr_done[kMaxDevices][2] = {};
+
+template <int D>
+zz_status_t ensure_smem_attr() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(ZZ_ERR_UNSUPPORTED, "device ordinal above 255");
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  bool& done = g_attr_done[dev][D == 128 ? 1 : 0];
+  if (!done) {
+    e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmem);
+    if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    done = true;
   }
-  return std::max(1, (sms + groups_per_kv - 1) / groups_per_kv);
+  return ZZ_OK;
 }
 
 template <int D>
@@ -610,12 +629,7 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: grid too large");
   p.n_items = int(n_items);
   p.chunk_items = chunk_items_for(p.groups_per_kv);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-    attr_set = true;
-  }
+  if (zz_status_t e = ensure_smem_attr<D>()) return e;
   attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));
@@ -629,29 +643,35 @@ bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) ==
 // Scratch of zz_attn_prefill_noalloc: the half table, the work list and the
 // status word live here instead of in a caller-allocated workspace.  Every GPU
 // that loads the library keeps this array until the process exits.
+// Layout: [status word (16 B) | pad to 256 | half table | pad to 256 | work items].
 constexpr size_t kStaticScratchBytes = size_t(1) << 20;   // 1 MiB
+constexpr size_t kStaticHalvesOff = 256;
 __device__ __align__(256) static unsigned char g_static_scratch[kStaticScratchBytes];
 
 std::mutex g_scratch_mu;
-void* g_scratch_addr[256] = {};   // device address of g_static_scratch, per device ordinal
+void* g_scratch_addr[kMaxDevices] = {};   // device address of g_static_scratch, per device ordinal
 
-// Device address of the static scratch on the current device.  The name of the
-// array is only a host-side stand-in; the address must come from the runtime.
-zz_status_t static_scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
-  if (dev < 0 || dev >= 256) return fail(ZZ_ERR_UNSUPPORTED, "device ordinal above 255");
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
-    if (e != cudaSuccess || !ptr)
-      return fail(ZZ_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-    g_scratch_addr[dev] = ptr;
-  }
-  *out = g_scratch_addr[dev];
-  return ZZ_OK;
+// The tables reach the static array as kernel parameters: the runtime copies a
+// launch's parameters into its command stream when the launch is enqueued, so
+// this needs neither a staging buffer (no host or device allocation) nor a
+// copy from pageable memory (which would wait for the stream).  One launch
+// carries up to kFillBytes; the first one also clears the status word.
+constexpr int kFillWords = 2040;
+constexpr uint32_t kFillBytes = kFillWords * 16;
+struct FillArgs {
+  uint32_t offset;        // destination byte offset in g_static_scratch (16-byte aligned)
+  uint32_t nbytes;        // bytes of data[] to store (a multiple of 16)
+  uint32_t clear_status;  // 1: also zero the 16-byte status word
+  uint32_t pad;
+  uint4 data[kFillWords];
+};
+static_assert(sizeof(FillArgs) <= 32764, "kernel parameters are limited to 32764 bytes");
+
+__global__ void __launch_bounds__(256) static_scratch_fill(const __grid_constant__ FillArgs a) {
+  uint4* dst = reinterpret_cast<uint4*>(g_static_scratch + a.offset);
+  for (uint32_t i = threadIdx.x; i < a.nbytes / 16; i += blockDim.x) dst[i] = a.data[i];
+  if (a.clear_status && threadIdx.x == 0)
+    *reinterpret_cast<uint4*>(g_static_scratch) = make_uint4(0u, 0u, 0u, 0u);
 }
 
 template <int D>
@@ -668,35 +688,35 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   const std::vector<int32_t>& off = pair_heads ? pl->tile_rank_off : pl->pair_rank_off;
   const size_t first = all ? 0 : size_t(off[rank_begin]);
   const size_t n_items = all ? list.size() : size_t(off[rank_begin + rank_count] - off[rank_begin]);
-  // Layout inside the static array: [status | halves | work items].
-  const size_t halves_off = 256;
   const size_t halves_bytes = pl->halves.size() * sizeof(HalfDesc);
-  const size_t items_off = (halves_off + halves_bytes + 255) & ~size_t(255);
-  const size_t need = items_off + n_items * sizeof(WorkItem);
+  const size_t items_off = (kStaticHalvesOff + halves_bytes + 255) & ~size_t(255);
+  const size_t items_bytes = n_items * sizeof(WorkItem);
+  const size_t need = items_off + items_bytes;
+  // ---- every check comes before anything is enqueued ----
   if (need > kStaticScratchBytes)
     return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: plan tables need " + std::to_string(need) +
                                         " bytes, more than the static scratch of " +
                                         std::to_string(kStaticScratchBytes) + " bytes");
+  if (num_slots > int64_t(INT32_MAX) - page_size)
+    return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: num_slots too large");
   if (n_items == 0) return ZZ_OK;
+  const int head_groups = pair_heads ? h_q / 2 : h_q;
+  const int64_t grid = int64_t(n_items) * head_groups;
+  if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: grid too large");
   if (zz_status_t e = get_encoder()) return e;
-  void* base = nullptr;
-  if (zz_status_t e = static_scratch_address(&base)) return e;
-  char* sc = static_cast<char*>(base);
-  cudaError_t e = cudaMemsetAsync(sc, 0, 16, stream);   // status word starts at zero
-  if (e == cudaSuccess && halves_bytes)
-    e = cudaMemcpyAsync(sc + halves_off, pl->halves.data(), halves_bytes, cudaMemcpyHostToDevice, stream);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(sc + items_off, list.data() + first, n_items * sizeof(WorkItem),
-                        cudaMemcpyHostToDevice, stream);
-  if (e != cudaSuccess)
-    return fail(ZZ_ERR_CUDA, std::string("zz_attn_prefill_noalloc: ") + cudaGetErrorString(e));
   const int box_rows = page_size >= 128 ? 128 : page_size;
   CUtensorMap tq, tk, tv;
   if (zz_status_t st = encode_3d(&tq, q, D, h_q, int64_t(rank_count) * pl->M, 128)) return st;
   if (zz_status_t st = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return st;
   if (zz_status_t st = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return st;
+  if (zz_status_t e = ensure_smem_attr<D>()) return e;
+  void* base = nullptr;
+  if (zz_status_t e = static_scratch_address(&base)) return e;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(ZZ_ERR_CUDA, "zz_attn_prefill_noalloc: cudaGetDevice");
+  char* sc = static_cast<char*>(base);
   Params p{};
-  p.halves = reinterpret_cast<const HalfDesc*>(sc + halves_off);
+  p.halves = reinterpret_cast<const HalfDesc*>(sc + kStaticHalvesOff);
   p.items = reinterpret_cast<const WorkItem*>(sc + items_off);
   p.status = reinterpret_cast<int*>(sc);
   p.page_table = page_table;
@@ -709,31 +729,87 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   p.h_kv = h_kv;
   p.group = group;
   p.pair_heads = pair_heads ? 1 : 0;
-  p.head_groups = pair_heads ? h_q / 2 : h_q;
+  p.head_groups = head_groups;
   p.groups_per_kv = pair_heads ? group / 2 : group;
   p.M = pl->M;
   p.rank_begin = rank_begin;
   p.max_pages = max_pages;
   p.page_size = page_size;
   p.box_rows = box_rows;
-  if (num_slots > int64_t(INT32_MAX) - page_size) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: num_slots too large");
   p.num_pages = int((num_slots + page_size - 1) / page_size);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = 1000000000ull;
   p.causal = 1;
-  const int64_t grid = int64_t(n_items) * p.head_groups;
-  if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: grid too large");
   p.n_items = int(n_items);
   p.chunk_items = chunk_items_for(p.groups_per_kv);
-  e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+  // ---- enqueue: the tables (in launches of up to kFillBytes), then the attention ----
+  // Bytes [kStaticHalvesOff, need) of the array's image: the half table, zeros
+  // up to items_off, then this call's work items.
+  const char* halves_src = reinterpret_cast<const char*>(pl->halves.data());
+  const char* items_src = reinterpret_cast<const char*>(list.data() + first);
+  FillArgs fa;
+  bool first_fill = true;
+  for (size_t at = kStaticHalvesOff; at < need; at += kFillBytes) {
+    const size_t len = std::min<size_t>(kFillBytes, need - at);
+    const size_t padded = (len + 15) & ~size_t(15);
+    char* dst = reinterpret_cast<char*>(fa.data);
+    std::memset(dst, 0, padded);
+    const size_t h_lo = std::max(at, kStaticHalvesOff), h_hi = std::min(at + len, kStaticHalvesOff + halves_bytes);
+    if (h_lo < h_hi) std::memcpy(dst + (h_lo - at), halves_src + (h_lo - kStaticHalvesOff), h_hi - h_lo);
+    const size_t i_lo = std::max(at, items_off), i_hi = std::min(at + len, need);
+    if (i_lo < i_hi) std::memcpy(dst + (i_lo - at), items_src + (i_lo - items_off), i_hi - i_lo);
+    fa.offset = uint32_t(at);
+    fa.nbytes = uint32_t(padded);
+    fa.clear_status = first_fill ? 1u : 0u;
+    fa.pad = 0;
+    static_scratch_fill<<<1, 256, 0, stream>>>(fa);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("static_scratch_fill launch: ") + cudaGetErrorString(e));
+    first_fill = false;
+  }
+  pl->noalloc_dev.store(dev);
   attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));
   return ZZ_OK;
 }
 
 }  // namespace
+
+// Device address of the static scratch on the current device.  In host code the
+// array's name is only a stand-in; the address must come from the runtime,
+// looked up once per device with that device current.
+zz_status_t static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(ZZ_ERR_UNSUPPORTED, "device ordinal above 255");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(ZZ_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return ZZ_OK;
+}
+
+std::mutex g_sm_mu;
+int g_sm_count[256] = {};
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 148;
+  std::lock_guard<std::mutex> lock(g_sm_mu);
+  if (!g_sm_count[dev]) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+    g_sm_count[dev] = sms;
+  }
+  return g_sm_count[dev];
+}
 }  // namespace zz
 
 extern "C" zz_status_t zz_attn_prefill_ex(const zz_plan_t* plan, int rank_begin, int rank_count,

@@ -1,6 +1,7 @@
 // Internal declarations shared by the host planner and the CUDA entry points.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <string>
 #include <vector>
@@ -64,9 +65,17 @@ struct zz_plan {
   zz::Workspace ws{};
   void* dev_ws = nullptr;
   void* staging = nullptr;   // pinned host image of the workspace, made at the first upload
+  // Device ordinal of the last zz_attn_prefill_noalloc call made with this plan
+  // (-1: none); zz_plan_device_status then also reads the static status word.
+  mutable std::atomic<int> noalloc_dev{-1};
 };
 
 namespace zz {
 zz_status_t fail(zz_status_t st, const std::string& msg);
 zz_status_t ok();
+// Device address of the allocation-free entry point's static scratch on the
+// current device (its first 16 bytes are that entry point's status word).
+zz_status_t static_scratch_address(void** out);
+// Streaming multiprocessors of the current device (cached per device ordinal).
+int device_sm_count();
 }  // namespace zz

@@ -369,14 +369,40 @@ extern "C" zz_status_t zz_plan_upload(zz_plan_t* p, void* dev, size_t bytes, voi
 extern "C" zz_status_t zz_plan_device_status(const zz_plan_t* p, int32_t* flags, int clear,
                                              void* stream) {
   if (!p || !flags) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_device_status: NULL argument");
-  if (!p->dev_ws) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_device_status: plan not uploaded");
+  const int noalloc_dev = p->noalloc_dev.load();
+  if (!p->dev_ws && noalloc_dev < 0)
+    return zz::fail(ZZ_ERR_INVALID_ARG,
+                    "zz_plan_device_status: plan neither uploaded nor used by zz_attn_prefill_noalloc");
   auto s = static_cast<cudaStream_t>(stream);
-  char* st = static_cast<char*>(p->dev_ws) + p->ws.status;
-  cudaError_t e = cudaMemcpyAsync(flags, st, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  // Status words to read: the plan's workspace word, and the static array's
+  // word when this plan's last allocation-free call ran on the current device.
+  char* words[2] = {nullptr, nullptr};
+  int n = 0;
+  if (p->dev_ws) words[n++] = static_cast<char*>(p->dev_ws) + p->ws.status;
+  if (noalloc_dev >= 0) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+      return zz::fail(ZZ_ERR_CUDA, std::string("zz_plan_device_status: ") + cudaGetErrorString(e));
+    if (dev == noalloc_dev) {
+      void* base = nullptr;
+      if (zz_status_t st = zz::static_scratch_address(&base)) return st;
+      words[n++] = static_cast<char*>(base);
+    } else if (!p->dev_ws) {
+      return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_device_status: make the device of the plan's last "
+                                          "zz_attn_prefill_noalloc call current first");
+    }
+  }
+  int32_t got[2] = {0, 0};
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < n && e == cudaSuccess; ++i)
+    e = cudaMemcpyAsync(&got[i], words[i], sizeof(int32_t), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e == cudaSuccess && clear) e = cudaMemsetAsync(st, 0, 4 * sizeof(int32_t), s);
+  for (int i = 0; i < n && e == cudaSuccess && clear; ++i)
+    e = cudaMemsetAsync(words[i], 0, 4 * sizeof(int32_t), s);
   if (e != cudaSuccess)
     return zz::fail(ZZ_ERR_CUDA, std::string("zz_plan_device_status: ") + cudaGetErrorString(e));
+  *flags = got[0] | got[1];
   if (*flags & zz::kStatusTimeout)
     return zz::fail(ZZ_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (pipeline stalled)");
   if (*flags & zz::kStatusBadPage)

@@ -664,7 +664,7 @@ def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 5
     """Attention (and rerange) kernel time on every configuration's shape.
 
     Per configuration: seeded inputs, plan, shard, rerange into the paged pool,
-    then ``reps`` timed launches of each kernel, each launch preceded by a write
+    then ``reps`` timed launches of each kernel, each launch preceded by a read
     of ``flush_mb`` MB (so every launch starts with a cold L2), each timed alone
     with CUDA events on the launching stream; the median is reported.  FLOPs
     are the exact causal pairs x 4 * D * H_q; rerange bytes are K and V, read
@@ -674,7 +674,7 @@ def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 5
     burst = float(peaks.get("bf16_tflops"))
     sus = float(peaks.get("bf16_tflops_sustained", burst))
     hbm = float(peaks["hbm_gbs"])
-    flush = torch.empty(flush_mb << 20, dtype=torch.uint8, device=dev)
+    flush = torch.ones((flush_mb << 20) // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
     out_rows = []
     for name, cp, spec, h_q, h_kv, d, ps, dtype, vscale, pseed in PER_CONFIG:
@@ -705,7 +705,7 @@ def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 5
         def timed(fn):
             ts = []
             for i in range(reps + 1):
-                flush.zero_()
+                flush.sum()              # a read: evicts L2 without leaving dirty lines behind
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 fn()
@@ -733,7 +733,7 @@ def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 5
     del flush
     torch.cuda.empty_cache()
     return {"rows": out_rows, "peak_source": f"{src} (burst: launches of at most ~0.25 s, timed alone)",
-            "method": f"median of {reps} launches per kernel, each after a {flush_mb} MB L2 flush, "
+            "method": f"median of {reps} launches per kernel, each after a {flush_mb} MB read (L2 flush), "
                       "CUDA events on the launching stream"}
 
 

@@ -40,6 +40,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "ptx_sm100.cuh"
 #include "exp2_poly.h"
@@ -64,11 +65,16 @@ constexpr int kWarpMma = 8;
 constexpr int kWarpLoad = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 256 between rescales
-// Of the 16 exponential pairs of each 32-column chunk, pairs >= kPolyFrom are
-// evaluated with the FMA-pipe polynomial, the rest with MUFU ex2.  Measured on
-// B200 with this pipeline, sending 25% to the polynomial (kPolyFrom = 12) was
-// ~5% slower than MUFU alone, so all pairs use ex2 (kPolyFrom = 16).
-constexpr int kPolyFrom = 16;
+// Bit e of kPolyMask: exponential pair e (of the 16 pairs of each 32-column
+// chunk of an S row) is evaluated with the FMA-pipe polynomial of exp2_poly.h
+// instead of MUFU ex2, on tiles that need no causal mask (masked tiles keep
+// ex2, whose 2^-inf is exactly 0).  Per K/V tile the MUFU work of both
+// softmax groups equals the tensor-core work, so moving a share of the
+// exponentials to the FMA pipe shortens each sub-tile's softmax.
+#ifndef ZZ_POLY_MASK
+#define ZZ_POLY_MASK 0u
+#endif
+constexpr uint32_t kPolyMask = ZZ_POLY_MASK;
 
 template <int D>
 struct Cfg {
@@ -408,7 +414,8 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
       // Causal mask, only on tiles that reach past the sub-tile's first row.
-      if (j * 128 + 127 > first_pos) {
+      const bool masked = j * 128 + 127 > first_pos;
+      if (masked) {
         const int limit = my_pos - j * 128 + 1;   // visible keys of this row in this tile
 #pragma unroll
         for (int c = 0; c < 128; ++c)
@@ -443,30 +450,34 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         m = m_tile;
       }
-      // P = 2^(s*scale*log2e - m): packed FMA, ex2, packed running sum, bf16
-      // pairs written over the first 64 columns of S.
+      // P = 2^(s*scale*log2e - m): packed FMA, ex2 (or the polynomial), packed
+      // running sum, bf16 pairs written over the first 64 columns of S.
       const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
       const float2 nm2 = make_float2(-m, -m);
       float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
+      auto exp_row = [&](auto use_poly) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int col = c * 32 + 2 * e;
-          float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2, nm2);
-          if (e >= kPolyFrom) {
-            x = exp2_poly2(x);
-          } else {
-            x.x = ex2(x.x);
-            x.y = ex2(x.y);
+          for (int e = 0; e < 16; ++e) {
+            const int col = c * 32 + 2 * e;
+            float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2, nm2);
+            if (decltype(use_poly)::value && ((kPolyMask >> e) & 1u)) {
+              x = exp2_poly2(x);
+            } else {
+              x.x = ex2(x.x);
+              x.y = ex2(x.y);
+            }
+            acc4[e & 3] = fadd2(acc4[e & 3], x);
+            pk[e] = pack_bf16x2(x.x, x.y);
           }
-          acc4[e & 3] = fadd2(acc4[e & 3], x);
-          pk[e] = pack_bf16x2(x.x, x.y);
+          tmem_st16(t_s + c * 16, pk);
         }
-        tmem_st16(t_s + c * 16, pk);
-      }
+      };
+      if (kPolyMask == 0u || masked) exp_row(std::false_type{});
+      else exp_row(std::true_type{});
       const float2 acc = fadd2(fadd2(acc4[0], acc4[1]), fadd2(acc4[2], acc4[3]));
       l += acc.x + acc.y;
       tmem_wait_st();

@@ -523,6 +523,405 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
 }
 
+// ---------------------------------------------------------------- CTA-pair kernel
+// attn_fwd_pair: the same attention with two CTAs per MMA (tcgen05 .cta_group::2),
+// for D = 128 and GQA groups that are multiples of 4.  A cluster of two CTAs
+// takes one work item and four query heads that share a K/V head: CTA rank r
+// owns heads 4q + 2r and 4q + 2r + 1 (its sub-tiles 0 and 1).  Each pair MMA
+// has M = 256 (128 rows from each CTA) and splits B by N across the pair, so
+// every CTA loads only half of each K tile (64 keys, all 128 dims) and half of
+// each V tile (all 128 keys, 64 dims): per SM, half the K/V bytes and half the
+// TMA boxes of the single-CTA kernel for the same FLOPs.  CTA 0 issues every
+// MMA; its commits arrive on the barriers of both CTAs.
+struct PairCfg {
+  static constexpr int kBoxBytes = 128 * 128;
+  static constexpr int kQBytes = 2 * kBoxBytes;           // Q tile: 128 rows x 128 dims
+  static constexpr int kKHalfBytes = 2 * 64 * 128;        // 64 keys x 128 dims (two 8 KB column boxes)
+  static constexpr int kVHalfBytes = 128 * 128;           // 128 keys x 64 dims (one box)
+  static constexpr int kStageBytes = kKHalfBytes + kVHalfBytes;
+  static constexpr int kStages = 5;
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kQBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kStageBytes;
+  static constexpr int kSmem = kBarOff + 512 + 1024;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
+};
+static_assert(PairCfg::kSmem <= 232448, "227 KB of shared memory per CTA");
+// setmaxnreg split of the pair kernel (the one without spills for its code).
+constexpr uint32_t kPairRegsSoftmax = 208, kPairRegsOther = 88;
+static_assert(2 * kPairRegsSoftmax + kPairRegsOther <= 3 * 168, "register split exceeds the launch's registers");
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using C = PairCfg;
+  constexpr int D = 128;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::kBarOff);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();     // 0: leader (issues the MMAs), 1: peer
+  const bool leader = rank == 0;
+
+  // ---- work decomposition: clusters in chunks of items, K/V-head-major ----
+  int item_idx, quad;
+  {
+    const int cl = blockIdx.x >> 1;
+    const int quads_per_kv = p.groups_per_kv >> 1;       // clusters per K/V head and item
+    const int per_chunk = p.chunk_items * (p.head_groups >> 1);
+    const int chunk = cl / per_chunk;
+    const int r = cl - chunk * per_chunk;
+    const int w_items = min(p.chunk_items, p.n_items - chunk * p.chunk_items);
+    const int kvh = r / (w_items * quads_per_kv);
+    const int r2 = r - kvh * w_items * quads_per_kv;
+    item_idx = chunk * p.chunk_items + r2 / quads_per_kv;
+    quad = kvh * quads_per_kv + r2 % quads_per_kv;
+  }
+  const WorkItem w = p.items[item_idx];
+  const HalfDesc hd = p.halves[w.half_id];
+  SubTile st[2];
+  st[0] = {4 * quad + 2 * int(rank), w.tile * 128, 0};
+  st[1] = {4 * quad + 2 * int(rank) + 1, w.tile * 128, 0};
+  st[0].n = tiles_for(hd, st[0].q0, p.causal);
+  st[1].n = st[0].n;                                     // same rows, same keys
+  const int kv_end = p.causal ? hd.kv_len : hd.kv_full;
+  const int n_max = st[0].n;
+  const int kv_head = st[0].head / p.group;
+  const int64_t row_base = int64_t(hd.rank - p.rank_begin) * p.M + hd.row0;
+
+  // ---- setup: barriers in both CTAs, TMEM for the pair, then a cluster barrier
+  // so that no CTA signals the other's barriers before they exist ----
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q_full[i], 2);      // one expect_tx arrival from each CTA's producer
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 256);    // 128 softmax threads of each CTA
+      mbar_init(&bars->o_full[i], 1);
+    }
+    mbar_init(&bars->mma_done, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 2);     // one expect_tx arrival from each CTA's producer
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    bars->abort = (p.status && (*reinterpret_cast<volatile int*>(p.status) & kStatusTimeout)) ? 1 : 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc_pair(&bars->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+    tc_fence_before();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  // The leader's barriers, as shared::cluster addresses (the peer signals them remotely).
+  const uint32_t lead_q_full0 = mapa_shared(smem_u32(&bars->q_full[0]), 0);
+  const uint32_t lead_kv_full0 = mapa_shared(smem_u32(&bars->kv_full[0]), 0);
+  const uint32_t lead_p_full0 = mapa_shared(smem_u32(&bars->p_full[0]), 0);
+
+  if (warp >= 8) {
+  regs_dec<kPairRegsOther>();
+  if (warp == kWarpLoad) {
+    // ================= TMA producer (both CTAs: this CTA's halves) =================
+    const int32_t* pt = p.page_table + int64_t(hd.seq) * p.max_pages;
+    bool q_issued[2] = {false, false};
+    if (lane == 0 && !*abort) {
+      for (int i = 0; i < 2; ++i) {
+        if (n_max == 0) continue;
+        q_issued[i] = true;
+        uint8_t* dst = smem + C::kQOff + i * C::kQBytes;
+        const uint32_t bar = lead_q_full0 + uint32_t(i) * 8u;
+        mbar_arrive_expect_tx_cluster(bar, C::kQBytes);
+        for (int b = 0; b < 2; ++b)
+          tma_load_3d_pair(dst + b * C::kBoxBytes, &tm_q, bar, b * 64, st[i].head, int32_t(row_base + st[i].q0));
+      }
+    }
+    const int kbox = p.box_rows < 64 ? p.box_rows : 64;       // K half: 64 keys
+    const int vbox = p.box_rows;                              // V half: 128 keys
+    const int kchunks = 64 / kbox, vchunks = 128 / vbox;
+    bool bad_page = false;
+    // Stage t (t = 0 .. n_max): this CTA's half of K_t if t < n_max, of V_{t-1} if t >= 1.
+    int t = 0;
+    for (; t <= n_max && !*abort; ++t) {
+      const int slot = t % C::kStages;
+      const uint32_t use = t / C::kStages;
+      if (!wait_parity(&bars->kv_empty[slot], (use & 1u) ^ 1u, abort, p.timeout_ns)) break;
+      uint8_t* stage = smem + C::kKVOff + slot * C::kStageBytes;
+      uint8_t* ktile = stage;
+      uint8_t* vtile = stage + C::kKHalfBytes;
+      const bool has_k = t < n_max, has_v = t >= 1;
+      const int key0k = t * 128 + 64 * int(rank);           // first key of this CTA's K half
+      const int key0v = (t - 1) * 128;                       // first key of the V tile
+      uint32_t tma_bytes = 0;
+      bool manual = false;
+      if (has_k)
+        for (int c = 0; c < kchunks; ++c) {
+          if (key0k + (c + 1) * kbox <= kv_end) tma_bytes += kbox * 128 * 2;
+          else manual = true;
+        }
+      if (has_v)
+        for (int c = 0; c < vchunks; ++c) {
+          if (key0v + (c + 1) * vbox <= kv_end) tma_bytes += vbox * 128;
+          else manual = true;
+        }
+      if (manual) {
+        // Rows at or beyond kv_len are filled by hand (real keys copied, the rest zero).
+        for (int which = 0; which < 2; ++which) {
+          if (which == 0 && !has_k) continue;
+          if (which == 1 && !has_v) continue;
+          const int rows = which == 0 ? 64 : 128, box = which == 0 ? kbox : vbox;
+          const int units_per_row = which == 0 ? 16 : 8;     // 16-byte pieces of this CTA's part of a row
+          const int key0 = which == 0 ? key0k : key0v;
+          const __nv_bfloat16* pool = which == 0 ? p.k_pool : p.v_pool;
+          for (int c = 0; c < rows / box; ++c) {
+            if (key0 + (c + 1) * box <= kv_end) continue;
+            for (int u = lane; u < box * units_per_row; u += 32) {
+              const int row = c * box + u / units_per_row;
+              const int rem = u % units_per_row;
+              const int b = rem >> 3, ch = rem & 7;          // column box (K only) and 16-byte piece
+              const int key = key0 + row;
+              const int col = which == 0 ? b * 64 + ch * 8 : 64 * int(rank) + ch * 8;
+              int4 v = make_int4(0, 0, 0, 0);
+              if (key < kv_end) {
+                const int64_t slot_id = int64_t(__ldg(pt + key / p.page_size)) * p.page_size + key % p.page_size;
+                if (slot_id >= 0 && slot_id < p.num_slots)
+                  v = __ldg(reinterpret_cast<const int4*>(pool + (slot_id * p.h_kv + kv_head) * D + col));
+                else
+                  bad_page = true;
+              }
+              uint8_t* dstp = which == 0 ? ktile + b * (64 * 128) : vtile;
+              *reinterpret_cast<int4*>(dstp + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      const uint32_t bar = lead_kv_full0 + uint32_t(slot) * 8u;
+      if (lane == 0) mbar_arrive_expect_tx_cluster(bar, tma_bytes);
+      __syncwarp();
+      // One lane per page chunk: K chunks first, then V chunks.
+      const int nk = has_k ? kchunks : 0, nv = has_v ? vchunks : 0;
+      for (int u = lane; u < nk + nv; u += 32) {
+        const bool is_k = u < nk;
+        const int c = is_k ? u : u - nk;
+        const int box = is_k ? kbox : vbox;
+        const int kc = (is_k ? key0k : key0v) + c * box;
+        if (kc + box > kv_end) continue;
+        const int32_t page = __ldg(pt + kc / p.page_size);
+        const bool in_pool = uint32_t(page) < uint32_t(p.num_pages);
+        bad_page |= !in_pool;
+        const int32_t slot0 = (in_pool ? page : p.num_pages) * p.page_size + kc % p.page_size;
+        if (is_k) {
+          for (int b = 0; b < 2; ++b)
+            tma_load_3d_pair(ktile + b * (64 * 128) + c * box * 128, &tm_k, bar, b * 64, kv_head, slot0);
+        } else {
+          tma_load_3d_pair(vtile + c * box * 128, &tm_v, bar, 64 * int(rank), kv_head, slot0);
+        }
+      }
+      __syncwarp();
+    }
+    const int load_no = t;
+    if (bad_page && p.status) atomicOr(p.status, kStatusBadPage);
+    // Copies of both CTAs land on the leader's barriers: the leader's producer
+    // drains them; the cluster barrier at the end keeps the peer alive until then.
+    if (lane == 0 && leader) {
+      for (int n = max(0, load_no - C::kStages); n < load_no; ++n)
+        drain_parity(&bars->kv_full[n % C::kStages], (uint32_t(n / C::kStages)) & 1u, p.timeout_ns);
+      for (int i = 0; i < 2; ++i)
+        if (q_issued[i]) drain_parity(&bars->q_full[i], 0, p.timeout_ns);
+    }
+  } else if (warp == kWarpMma && leader) {
+    // ================= MMA issue (leader CTA, one thread) =================
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(256, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(256, D, false, true);
+      const uint32_t kv_addr = smem_u32(smem + C::kKVOff);
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+      const uint64_t dq1 = dq0 + uint64_t(C::kQBytes >> 4);
+      const uint64_t dk0 = smem_desc_sw128(kv_addr, 16, 1024);                       // K half of stage 0
+      const uint64_t dv0 = smem_desc_sw128(kv_addr + C::kKHalfBytes, 16, 1024);      // V half of stage 0
+      const uint16_t both = 3;
+      auto issue_s = [&](uint32_t col, uint64_t dq, int slot) {
+        const uint64_t dk = dk0 + uint64_t((slot * C::kStageBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qoff = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+          const uint32_t koff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
+          mma_ss_pair(tmem + col, dq + qoff, dk + koff, idesc_s, kk > 0);
+        }
+      };
+      auto issue_pv = [&](uint32_t col_o, uint32_t col_p, int slot, bool acc) {
+        const uint64_t dv = dv0 + uint64_t((slot * C::kStageBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts_pair(tmem + col_o, tmem + col_p + kk * 8, dv + uint64_t((kk * 2048) >> 4), idesc_o,
+                      (acc || kk > 0) ? 1u : 0u);
+      };
+      const int n = n_max;
+      bool ok = n > 0;
+      if (ok) ok = wait_parity(&bars->q_full[0], 0, abort, p.timeout_ns);
+      if (ok) ok = wait_parity(&bars->q_full[1], 0, abort, p.timeout_ns);
+      if (ok) ok = wait_parity(&bars->kv_full[0], 0, abort, p.timeout_ns);   // stage 0: K_0
+      if (ok) {
+        tc_fence_after();
+        issue_s(C::kColS0, dq0, 0); mma_commit_pair(&bars->s_full[0], both);
+        issue_s(C::kColS1, dq1, 0); mma_commit_pair(&bars->s_full[1], both);
+        mma_commit_pair(&bars->kv_empty[0], both);
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int t = j + 1;                    // stage with V_j and K_{j+1}
+        const int slot = t % C::kStages;
+        if (!(ok = wait_parity(&bars->kv_full[slot], uint32_t(t / C::kStages) & 1u, abort, p.timeout_ns))) break;
+        if (!(ok = wait_parity(&bars->p_full[0], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+        tc_fence_after();
+        issue_pv(C::kColO0, C::kColS0, slot, j > 0);
+        if (j == n - 1) mma_commit_pair(&bars->o_full[0], both);
+        else { issue_s(C::kColS0, dq0, slot); mma_commit_pair(&bars->s_full[0], both); }
+        if (!(ok = wait_parity(&bars->p_full[1], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+        tc_fence_after();
+        issue_pv(C::kColO1, C::kColS1, slot, j > 0);
+        if (j == n - 1) mma_commit_pair(&bars->o_full[1], both);
+        else { issue_s(C::kColS1, dq1, slot); mma_commit_pair(&bars->s_full[1], both); }
+        mma_commit_pair(&bars->kv_empty[slot], both);
+      }
+      mma_commit_pair(&bars->mma_done, 1);
+      drain_parity(&bars->mma_done, 0, p.timeout_ns);
+    }
+    __syncwarp();
+  }   // the peer's MMA warp and warps 10-11 have no role here
+  } else {
+    // ================= softmax + epilogue (warps 0-7, both CTAs) =================
+    regs_inc<kPairRegsSoftmax>();
+    const int g = warp >> 2;
+    const SubTile& me = st[g];
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + (g ? C::kColS1 : C::kColS0);
+    const uint32_t t_o = tmem + lane_off + (g ? C::kColO1 : C::kColO0);
+    const uint32_t p_full_lead = lead_p_full0 + uint32_t(g) * 8u;
+    const int q_row = me.q0 + r;
+    const int my_pos = p.causal ? hd.kv_pos0 + q_row : hd.kv_full - 1;
+    const int first_pos = p.causal ? hd.kv_pos0 + me.q0 : hd.kv_full - 1;
+    float m = -CUDART_INF_F, l = 0.f;
+    bool ok = me.n > 0;
+    for (int j = 0; j < me.n && ok; ++j) {
+      if (!(ok = wait_parity(&bars->s_full[g], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+      tc_fence_after();
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_wait_ld();
+      const bool masked = j * 128 + 127 > first_pos;
+      if (masked) {
+        const int limit = my_pos - j * 128 + 1;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= limit) sr[c] = 0xFF800000u;
+      }
+      float pm[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) pm[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
+#pragma unroll
+      for (int c = 16; c < 128; c += 16)
+#pragma unroll
+        for (int q = 0; q < 8; q += 2)
+          pm[q] = fmax3(pm[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + q + 8])),
+          pm[q + 1] = fmax3(pm[q + 1], __uint_as_float(sr[c + q + 1]), __uint_as_float(sr[c + q + 9]));
+      const float mx = fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], fmax3(pm[5], pm[6], pm[7])));
+      const float m_tile = mx * p.scale_log2;
+      if (j == 0) {
+        m = m_tile;
+      } else if (m_tile > m + kRescaleThreshold) {
+        // S(j) completing implies P.V(j-1) completed: O is stable here.
+        const float f = ex2(m - m_tile);
+        l *= f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+          tmem_st32(t_o + c * 32, o);
+        }
+        m = m_tile;
+      }
+      const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nm2 = make_float2(-m, -m);
+      float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int col = c * 32 + 2 * e;
+          float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2, nm2);
+          x.x = ex2(x.x);
+          x.y = ex2(x.y);
+          acc4[e & 3] = fadd2(acc4[e & 3], x);
+          pk[e] = pack_bf16x2(x.x, x.y);
+        }
+        tmem_st16(t_s + c * 16, pk);
+      }
+      const float2 acc = fadd2(fadd2(acc4[0], acc4[1]), fadd2(acc4[2], acc4[3]));
+      l += acc.x + acc.y;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_cluster(p_full_lead);         // the leader's barrier, from either CTA
+    }
+    if (ok) ok = wait_parity(&bars->o_full[g], 0, abort, p.timeout_ns);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = q_row < hd.lq;
+      const int64_t grow = row_base + q_row;
+      const float inv = 1.f / l;
+      __nv_bfloat16* op = p.out + (grow * p.h_q + me.head) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        if (valid) {
+          int4* dst = reinterpret_cast<int4*>(op + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_int4(int(pk[4 * v]), int(pk[4 * v + 1]), int(pk[4 * v + 2]), int(pk[4 * v + 3]));
+        }
+      }
+      if (valid && p.lse) p.lse[grow * p.h_q + me.head] = (m + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  // ---- teardown: both CTAs done with TMEM and with each other's barriers ----
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && bars->abort && p.status) {
+    atomicOr(p.status, kStatusTimeout);
+    __threadfence();
+  }
+}
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -583,6 +982,54 @@ zz_status_t ensure_smem_attr() {
   return ZZ_OK;
 }
 
+// The CTA-pair kernel serves D = 128 with GQA groups that are multiples of 4
+// (four query heads of one K/V head per cluster); everything else runs the
+// single-CTA kernel.
+bool use_pair_kernel(int d, int group) { return d == 128 && group % 4 == 0; }
+
+std::mutex g_pair_attr_mu;
+bool g_pair_attr_done[256] = {};
+
+zz_status_t ensure_pair_attr() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 256) return fail(ZZ_ERR_UNSUPPORTED, "device ordinal above 255");
+  std::lock_guard<std::mutex> lock(g_pair_attr_mu);
+  if (!g_pair_attr_done[dev]) {
+    e = cudaFuncSetAttribute(attn_fwd_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmem);
+    if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    g_pair_attr_done[dev] = true;
+  }
+  return ZZ_OK;
+}
+
+// Tensor maps of the pair kernel (K boxes of at most 64 rows: a CTA loads 64
+// keys of each K tile) and its one-time attribute; enqueues nothing.
+zz_status_t prepare_pair(const void* q, int64_t q_rows, const void* k_pool, const void* v_pool,
+                         int64_t num_slots, int h_q, int h_kv, int page_size, CUtensorMap* tq,
+                         CUtensorMap* tk, CUtensorMap* tv, Params& p) {
+  if (zz_status_t e = get_encoder()) return e;
+  const int vbox = page_size >= 128 ? 128 : page_size;
+  const int kbox = vbox < 64 ? vbox : 64;
+  if (zz_status_t e = encode_3d(tq, q, 128, h_q, q_rows, 128)) return e;
+  if (zz_status_t e = encode_3d(tk, k_pool, 128, h_kv, num_slots, kbox)) return e;
+  if (zz_status_t e = encode_3d(tv, v_pool, 128, h_kv, num_slots, vbox)) return e;
+  if (zz_status_t e = ensure_pair_attr()) return e;
+  p.box_rows = vbox;
+  p.chunk_items = chunk_items_for(p.groups_per_kv);
+  return ZZ_OK;
+}
+
+// One CTA per head pair and work item; clusters of two CTAs along x.
+zz_status_t enqueue_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, int64_t grid,
+                         const Params& p, cudaStream_t stream) {
+  attn_fwd_pair<<<unsigned(grid), kThreads, PairCfg::kSmem, stream>>>(tq, tk, tv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_pair launch: ") + cudaGetErrorString(e));
+  return ZZ_OK;
+}
+
 template <int D>
 zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, const void* q,
                         const void* k_pool, const void* v_pool, int64_t num_slots,
@@ -639,6 +1086,12 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
   if (grid == 0) return ZZ_OK;
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: grid too large");
   p.n_items = int(n_items);
+  if (use_pair_kernel(D, p.group)) {
+    CUtensorMap pq, pk, pv;
+    if (zz_status_t e = prepare_pair(q, q_rows, k_pool, v_pool, num_slots, h_q, h_kv, page_size, &pq, &pk, &pv, p))
+      return e;
+    return enqueue_pair(pq, pk, pv, grid, p, stream);
+  }
   p.chunk_items = chunk_items_for(p.groups_per_kv);
   if (zz_status_t e = ensure_smem_attr<D>()) return e;
   attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
@@ -720,7 +1173,9 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   if (zz_status_t st = encode_3d(&tq, q, D, h_q, int64_t(rank_count) * pl->M, 128)) return st;
   if (zz_status_t st = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return st;
   if (zz_status_t st = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return st;
-  if (zz_status_t e = ensure_smem_attr<D>()) return e;
+  const bool pair = use_pair_kernel(D, group);
+  if (!pair)
+    if (zz_status_t e = ensure_smem_attr<D>()) return e;
   void* base = nullptr;
   if (zz_status_t e = static_scratch_address(&base)) return e;
   int dev = 0;
@@ -753,6 +1208,10 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   p.causal = 1;
   p.n_items = int(n_items);
   p.chunk_items = chunk_items_for(p.groups_per_kv);
+  if (pair)
+    if (zz_status_t e = prepare_pair(q, int64_t(rank_count) * pl->M, k_pool, v_pool, num_slots, h_q, h_kv,
+                                     page_size, &tq, &tk, &tv, p))
+      return e;
   // ---- enqueue: the tables (in launches of up to kFillBytes), then the attention ----
   // Bytes [kStaticHalvesOff, need) of the array's image: the half table, zeros
   // up to items_off, then this call's work items.
@@ -779,6 +1238,7 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
     first_fill = false;
   }
   pl->noalloc_dev.store(dev);
+  if (pair) return enqueue_pair(tq, tk, tv, grid, p, stream);
   attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));

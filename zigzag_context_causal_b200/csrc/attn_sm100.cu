@@ -30,6 +30,11 @@
 // other group's MMAs.  The softmax keeps a running maximum in log2 units and
 // only rescales O (in TMEM) when the maximum grows by more than 8, so most
 // tiles skip the correction.  Tiles past the causal diagonal are never loaded.
+//
+// attn_fwd_pair (further down) is the same pipeline on clusters of two CTAs
+// whose MMAs are shared (tcgen05 .cta_group::2, M = 256), for head_dim 128 and
+// GQA groups that are multiples of 4: per SM it loads half the K/V bytes and
+// issues half the TMA boxes, which is what bounds small pages.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>

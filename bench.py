@@ -616,7 +616,7 @@ def main_gpu(args):
         "attn_per_clock": per_clock(attn_tflops, clocks),
         "rerange_standalone": rerange_sweep,
         "per_config": per_config,
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_sm100", "achieved": attn_tflops,
+        "roofline": {"bound": "tensor", "kernel": attn_kernel_name(d, h_q, h_kv), "achieved": attn_tflops,
                      "peak": peak_sus, "unit": "TFLOP/s", "frac": attn_tflops / peak_sus,
                      "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel runs inside a long step)",
                      "traffic": traffic},
@@ -636,6 +636,12 @@ def main_gpu(args):
 # 524288 FLOPs, every 64 cycles), and the SM count.
 TENSOR_FLOP_PER_SM_CYCLE = 8192
 B200_SMS = 148
+
+
+def attn_kernel_name(d: int, h_q: int, h_kv: int) -> str:
+    """The attention kernel libzz runs for these shapes (bf16): CTA pairs for
+    head_dim 128 and GQA groups that are multiples of 4, single CTAs otherwise."""
+    return "attn_fwd_pair" if d == 128 and (h_q // h_kv) % 4 == 0 else "attn_fwd_sm100"
 
 
 def per_clock(tflops: float, clocks: dict):
@@ -739,6 +745,7 @@ def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 5
 
 KERNEL_SOURCES = {
     "attn_fwd_sm100": ["attn_sm100.cu", "ptx_sm100.cuh", "exp2_poly.h", "zz_internal.h"],
+    "attn_fwd_pair": ["attn_sm100.cu", "ptx_sm100.cuh", "exp2_poly.h", "zz_internal.h"],
     "rerange_standalone": ["rerange.cu", "zz_internal.h"],
     "push_rows": ["push.cu", "zz_internal.h"],
 }

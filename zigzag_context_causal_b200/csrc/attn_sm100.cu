@@ -411,7 +411,8 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = me.n > 0;
     for (int j = 0; j < me.n && ok; ++j) {
-      if (!(ok = wait_parity(&bars->s_full[g], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+      ok = wait_parity(&bars->s_full[g], uint32_t(j) & 1u, abort, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // TMEM access below is warp-wide
       tc_fence_after();
       // The whole 128-column row of S in registers: four loads, one wait.
       uint32_t sr[128];
@@ -440,20 +441,28 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const float m_tile = mx * p.scale_log2;
       if (j == 0) {
         m = m_tile;
-      } else if (m_tile > m + kRescaleThreshold) {
-        // S(j) completing implies P.V(j-1) completed: O is stable here.
-        const float f = ex2(m - m_tile);
-        l *= f;
+      } else {
+        // Rescale when the maximum grows by more than the threshold.  The TMEM
+        // loads and stores are warp-wide, so the whole warp takes the branch
+        // when any of its rows needs it; rows that keep their maximum use a
+        // factor of exactly 1.  S(j) completing implies P.V(j-1) completed:
+        // O is stable here.
+        const bool need = m_tile > m + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? m_tile : m;
+          const float f = ex2(m - m_new);
+          l *= f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_o + c * 32, o);
-          tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-          tmem_st32(t_o + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(t_o + c * 32, o);
+          }
+          m = m_new;
         }
-        m = m_tile;
       }
       // P = 2^(s*scale*log2e - m): packed FMA, ex2 (or the polynomial), packed
       // running sum, bf16 pairs written over the first 64 columns of S.
@@ -490,6 +499,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_arrive(&bars->p_full[g]);
     }
     if (ok) ok = wait_parity(&bars->o_full[g], 0, abort, p.timeout_ns);
+    ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-wide
     if (ok) {
       tc_fence_after();
       const bool valid = q_row < hd.lq;
@@ -821,7 +831,8 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = me.n > 0;
     for (int j = 0; j < me.n && ok; ++j) {
-      if (!(ok = wait_parity(&bars->s_full[g], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+      ok = wait_parity(&bars->s_full[g], uint32_t(j) & 1u, abort, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // TMEM access below is warp-wide
       tc_fence_after();
       uint32_t sr[128];
 #pragma unroll
@@ -847,20 +858,28 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const float m_tile = mx * p.scale_log2;
       if (j == 0) {
         m = m_tile;
-      } else if (m_tile > m + kRescaleThreshold) {
-        // S(j) completing implies P.V(j-1) completed: O is stable here.
-        const float f = ex2(m - m_tile);
-        l *= f;
+      } else {
+        // Rescale when the maximum grows by more than the threshold.  The TMEM
+        // loads and stores are warp-wide, so the whole warp takes the branch
+        // when any of its rows needs it; rows that keep their maximum use a
+        // factor of exactly 1.  S(j) completing implies P.V(j-1) completed:
+        // O is stable here.
+        const bool need = m_tile > m + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? m_tile : m;
+          const float f = ex2(m - m_new);
+          l *= f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_o + c * 32, o);
-          tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-          tmem_st32(t_o + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(t_o + c * 32, o);
+          }
+          m = m_new;
         }
-        m = m_tile;
       }
       const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
       const float2 nm2 = make_float2(-m, -m);
@@ -887,6 +906,7 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_arrive_cluster(p_full_lead);         // the leader's barrier, from either CTA
     }
     if (ok) ok = wait_parity(&bars->o_full[g], 0, abort, p.timeout_ns);
+    ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-wide
     if (ok) {
       tc_fence_after();
       const bool valid = q_row < hd.lq;

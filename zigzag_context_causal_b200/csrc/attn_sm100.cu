@@ -32,9 +32,9 @@
 // tiles skip the correction.  Tiles past the causal diagonal are never loaded.
 //
 // attn_fwd_pair (further down) is the same pipeline on clusters of two CTAs
-// whose MMAs are shared (tcgen05 .cta_group::2, M = 256), for head_dim 128 and
-// GQA groups that are multiples of 4: per SM it loads half the K/V bytes and
-// issues half the TMA boxes, which is what bounds small pages.
+// whose MMAs are shared (tcgen05 .cta_group::2, M = 256), for head_dim 128:
+// per SM it loads half the K/V bytes and issues half the TMA boxes, which is
+// what bounds small pages.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -119,6 +119,7 @@ struct Params {
   float scale_log2;
   uint64_t timeout_ns;
   int causal;           // 0: every row of a half sees all kv_full keys of its sequence
+  int pair_rows;        // CTA-pair kernel: 1 = four row tiles of one head per cluster, 0 = four heads
 };
 
 struct Bars {
@@ -540,9 +541,11 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 // ---------------------------------------------------------------- CTA-pair kernel
 // attn_fwd_pair: the same attention with two CTAs per MMA (tcgen05 .cta_group::2),
-// for D = 128 and GQA groups that are multiples of 4.  A cluster of two CTAs
-// takes one work item and four query heads that share a K/V head: CTA rank r
-// owns heads 4q + 2r and 4q + 2r + 1 (its sub-tiles 0 and 1).  Each pair MMA
+// for D = 128.  A cluster of two CTAs takes four 128-row sub-tiles that share a
+// K/V head: with a GQA group that is a multiple of 4, the same row tile of four
+// query heads (CTA rank r owns heads 4u + 2r and 4u + 2r + 1); otherwise four
+// consecutive row tiles of one head (CTA rank r owns tiles 4t + 2r and
+// 4t + 2r + 1), all run to the keys of the last one.  Each pair MMA
 // has M = 256 (128 rows from each CTA) and splits B by N across the pair, so
 // every CTA loads only half of each K tile (64 keys, all 128 dims) and half of
 // each V tile (all 128 keys, 64 dims): per SM, half the K/V bytes and half the
@@ -582,28 +585,43 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const bool leader = rank == 0;
 
   // ---- work decomposition: clusters in chunks of items, K/V-head-major ----
-  int item_idx, quad;
+  // Heads mode (GQA group a multiple of 4): a unit is a quad of query heads of
+  // one K/V head and one row tile; CTA rank r takes heads 4u + 2r, 4u + 2r + 1.
+  // Rows mode (any other group): a unit is one query head and a quad of row
+  // tiles; CTA rank r takes row tiles 4t + 2r and 4t + 2r + 1.
+  int item_idx, unit;
   {
     const int cl = blockIdx.x >> 1;
-    const int quads_per_kv = p.groups_per_kv >> 1;       // clusters per K/V head and item
-    const int per_chunk = p.chunk_items * (p.head_groups >> 1);
+    const int units_per_kv = p.pair_rows ? p.group : (p.groups_per_kv >> 1);
+    const int per_chunk = p.chunk_items * (p.pair_rows ? p.h_q : (p.head_groups >> 1));
     const int chunk = cl / per_chunk;
     const int r = cl - chunk * per_chunk;
     const int w_items = min(p.chunk_items, p.n_items - chunk * p.chunk_items);
-    const int kvh = r / (w_items * quads_per_kv);
-    const int r2 = r - kvh * w_items * quads_per_kv;
-    item_idx = chunk * p.chunk_items + r2 / quads_per_kv;
-    quad = kvh * quads_per_kv + r2 % quads_per_kv;
+    const int kvh = r / (w_items * units_per_kv);
+    const int r2 = r - kvh * w_items * units_per_kv;
+    item_idx = chunk * p.chunk_items + r2 / units_per_kv;
+    unit = kvh * units_per_kv + r2 % units_per_kv;
   }
   const WorkItem w = p.items[item_idx];
   const HalfDesc hd = p.halves[w.half_id];
   SubTile st[2];
-  st[0] = {4 * quad + 2 * int(rank), w.tile * 128, 0};
-  st[1] = {4 * quad + 2 * int(rank) + 1, w.tile * 128, 0};
-  st[0].n = tiles_for(hd, st[0].q0, p.causal);
-  st[1].n = st[0].n;                                     // same rows, same keys
+  int n_all;   // K/V tiles every sub-tile of the cluster visits (they share each MMA)
+  if (p.pair_rows) {
+    st[0] = {unit, (4 * w.tile + 2 * int(rank)) * 128, 0};
+    st[1] = {unit, (4 * w.tile + 2 * int(rank) + 1) * 128, 0};
+    // the keys of the quad's last valid row tile; lower rows see the extra
+    // tiles fully masked (P = 0), rows past the half are computed and not written
+    const int last_tile = min(4 * w.tile + 3, (hd.lq - 1) / 128);
+    n_all = tiles_for(hd, last_tile * 128, p.causal);
+  } else {
+    st[0] = {4 * unit + 2 * int(rank), w.tile * 128, 0};
+    st[1] = {4 * unit + 2 * int(rank) + 1, w.tile * 128, 0};
+    n_all = tiles_for(hd, st[0].q0, p.causal);            // same rows, same keys
+  }
+  st[0].n = n_all;
+  st[1].n = n_all;
   const int kv_end = p.causal ? hd.kv_len : hd.kv_full;
-  const int n_max = st[0].n;
+  const int n_max = n_all;
   const int kv_head = st[0].head / p.group;
   const int64_t row_base = int64_t(hd.rank - p.rank_begin) * p.M + hd.row0;
 
@@ -1007,10 +1025,52 @@ zz_status_t ensure_smem_attr() {
   return ZZ_OK;
 }
 
-// The CTA-pair kernel serves D = 128 with GQA groups that are multiples of 4
-// (four query heads of one K/V head per cluster); everything else runs the
-// single-CTA kernel.
-bool use_pair_kernel(int d, int group) { return d == 128 && group % 4 == 0; }
+// Which bf16 kernel a launch runs.  head_dim 128 runs on CTA pairs: four query
+// heads of one K/V head per cluster when the GQA group is a multiple of 4,
+// otherwise four row tiles of one head.  head_dim 64 runs on single CTAs.
+enum KernelChoice { kSingleCta = 0, kPairHeads = 1, kPairRows = 2 };
+KernelChoice kernel_for(int d, int group) {
+  if (d != 128) return kSingleCta;
+  return group % 4 == 0 ? kPairHeads : kPairRows;
+}
+
+// The plan's work list for a launch of ranks [rank_begin, rank_begin + rank_count):
+// row tiles (head pairs / head quads), row-tile pairs (single CTA, odd groups)
+// or row-tile quads (CTA pairs, rows mode).
+struct ItemRange {
+  const std::vector<WorkItem>* list;   // host copy
+  size_t ws_off;                       // its section in the plan workspace
+  size_t first, n;                     // first item and item count of the launch
+};
+ItemRange items_for(const zz_plan_t* pl, KernelChoice k, bool pair_heads, int rank_begin, int rank_count) {
+  const bool all = rank_count == pl->c;
+  const std::vector<WorkItem>* l_all;
+  const std::vector<WorkItem>* l_rank;
+  const std::vector<int32_t>* off;
+  size_t o_all, o_rank;
+  if (k == kPairRows) {
+    l_all = &pl->quads_all; l_rank = &pl->quads_rank; off = &pl->quad_rank_off;
+    o_all = pl->ws.quads_all; o_rank = pl->ws.quads_rank;
+  } else if (pair_heads) {
+    l_all = &pl->tiles_all; l_rank = &pl->tiles_rank; off = &pl->tile_rank_off;
+    o_all = pl->ws.tiles_all; o_rank = pl->ws.tiles_rank;
+  } else {
+    l_all = &pl->pairs_all; l_rank = &pl->pairs_rank; off = &pl->pair_rank_off;
+    o_all = pl->ws.pairs_all; o_rank = pl->ws.pairs_rank;
+  }
+  ItemRange r;
+  r.list = all ? l_all : l_rank;
+  r.ws_off = all ? o_all : o_rank;
+  r.first = all ? 0 : size_t((*off)[rank_begin]);
+  r.n = all ? l_all->size() : size_t((*off)[rank_begin + rank_count] - (*off)[rank_begin]);
+  return r;
+}
+
+// CTAs of a launch over n work items.
+int64_t grid_for(KernelChoice k, bool pair_heads, int64_t n, int h_q) {
+  if (k == kPairRows) return n * h_q * 2;
+  return n * (pair_heads ? h_q / 2 : h_q);
+}
 
 std::mutex g_pair_attr_mu;
 bool g_pair_attr_done[256] = {};
@@ -1042,11 +1102,14 @@ zz_status_t prepare_pair(const void* q, int64_t q_rows, const void* k_pool, cons
   if (zz_status_t e = encode_3d(tv, v_pool, 128, h_kv, num_slots, vbox)) return e;
   if (zz_status_t e = ensure_pair_attr()) return e;
   p.box_rows = vbox;
-  p.chunk_items = chunk_items_for(p.groups_per_kv);
+  // Items per scheduling chunk: one K/V head's CTAs of a chunk fill every SM
+  // once (rows mode: 2 x group CTAs per K/V head and item).
+  p.chunk_items = p.pair_rows ? std::max(1, (device_sm_count() + 2 * p.group - 1) / (2 * p.group))
+                              : chunk_items_for(p.groups_per_kv);
   return ZZ_OK;
 }
 
-// One CTA per head pair and work item; clusters of two CTAs along x.
+// Clusters of two CTAs along x (grid from grid_for).
 zz_status_t enqueue_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, int64_t grid,
                          const Params& p, cudaStream_t stream) {
   attn_fwd_pair<<<unsigned(grid), kThreads, PairCfg::kSmem, stream>>>(tq, tk, tv, p);
@@ -1061,13 +1124,8 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
                         const int32_t* page_table, int max_pages, int page_size, void* out,
                         float* lse, int h_q, int h_kv, float scale, int causal, cudaStream_t stream) {
   using C = Cfg<D>;
-  if (zz_status_t e = get_encoder()) return e;
   const int box_rows = page_size >= 128 ? 128 : page_size;
-  CUtensorMap tq, tk, tv;
   const int64_t q_rows = int64_t(rank_count) * pl->M;
-  if (zz_status_t e = encode_3d(&tq, q, D, h_q, q_rows, 128)) return e;
-  if (zz_status_t e = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return e;
-  if (zz_status_t e = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return e;
   const char* ws = static_cast<const char*>(pl->dev_ws);
   Params p{};
   p.halves = reinterpret_cast<const HalfDesc*>(ws + pl->ws.halves);
@@ -1094,29 +1152,25 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = 1000000000ull;   // 1 s per wait
   p.causal = causal;
-  int64_t n_items;
-  const bool all = rank_count == pl->c;
-  if (p.pair_heads) {
-    p.items = reinterpret_cast<const WorkItem*>(ws + (all ? pl->ws.tiles_all : pl->ws.tiles_rank)) +
-              (all ? 0 : pl->tile_rank_off[rank_begin]);
-    n_items = all ? int64_t(pl->tiles_all.size())
-                  : pl->tile_rank_off[rank_begin + rank_count] - pl->tile_rank_off[rank_begin];
-  } else {
-    p.items = reinterpret_cast<const WorkItem*>(ws + (all ? pl->ws.pairs_all : pl->ws.pairs_rank)) +
-              (all ? 0 : pl->pair_rank_off[rank_begin]);
-    n_items = all ? int64_t(pl->pairs_all.size())
-                  : pl->pair_rank_off[rank_begin + rank_count] - pl->pair_rank_off[rank_begin];
-  }
-  const int64_t grid = n_items * p.head_groups;
+  const KernelChoice kc = kernel_for(D, p.group);
+  p.pair_rows = kc == kPairRows ? 1 : 0;
+  const ItemRange ir = items_for(pl, kc, p.pair_heads != 0, rank_begin, rank_count);
+  p.items = reinterpret_cast<const WorkItem*>(ws + ir.ws_off) + ir.first;
+  const int64_t grid = grid_for(kc, p.pair_heads != 0, int64_t(ir.n), h_q);
   if (grid == 0) return ZZ_OK;
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill: grid too large");
-  p.n_items = int(n_items);
-  if (use_pair_kernel(D, p.group)) {
+  p.n_items = int(ir.n);
+  if (kc != kSingleCta) {
     CUtensorMap pq, pk, pv;
     if (zz_status_t e = prepare_pair(q, q_rows, k_pool, v_pool, num_slots, h_q, h_kv, page_size, &pq, &pk, &pv, p))
       return e;
     return enqueue_pair(pq, pk, pv, grid, p, stream);
   }
+  if (zz_status_t e = get_encoder()) return e;
+  CUtensorMap tq, tk, tv;
+  if (zz_status_t e = encode_3d(&tq, q, D, h_q, q_rows, 128)) return e;
+  if (zz_status_t e = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return e;
+  if (zz_status_t e = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return e;
   p.chunk_items = chunk_items_for(p.groups_per_kv);
   if (zz_status_t e = ensure_smem_attr<D>()) return e;
   attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
@@ -1171,12 +1225,11 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   using C = Cfg<D>;
   const int group = h_q / h_kv;
   const bool pair_heads = group % 2 == 0;
-  const bool all = rank_count == pl->c;
-  const std::vector<WorkItem>& list = pair_heads ? (all ? pl->tiles_all : pl->tiles_rank)
-                                                 : (all ? pl->pairs_all : pl->pairs_rank);
-  const std::vector<int32_t>& off = pair_heads ? pl->tile_rank_off : pl->pair_rank_off;
-  const size_t first = all ? 0 : size_t(off[rank_begin]);
-  const size_t n_items = all ? list.size() : size_t(off[rank_begin + rank_count] - off[rank_begin]);
+  const KernelChoice kc = kernel_for(D, group);
+  const ItemRange ir = items_for(pl, kc, pair_heads, rank_begin, rank_count);
+  const std::vector<WorkItem>& list = *ir.list;
+  const size_t first = ir.first;
+  const size_t n_items = ir.n;
   const size_t halves_bytes = pl->halves.size() * sizeof(HalfDesc);
   const size_t items_off = (kStaticHalvesOff + halves_bytes + 255) & ~size_t(255);
   const size_t items_bytes = n_items * sizeof(WorkItem);
@@ -1190,7 +1243,7 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
     return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: num_slots too large");
   if (n_items == 0) return ZZ_OK;
   const int head_groups = pair_heads ? h_q / 2 : h_q;
-  const int64_t grid = int64_t(n_items) * head_groups;
+  const int64_t grid = grid_for(kc, pair_heads, int64_t(n_items), h_q);
   if (grid > INT32_MAX) return fail(ZZ_ERR_INVALID_ARG, "zz_attn_prefill_noalloc: grid too large");
   if (zz_status_t e = get_encoder()) return e;
   const int box_rows = page_size >= 128 ? 128 : page_size;
@@ -1198,7 +1251,7 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   if (zz_status_t st = encode_3d(&tq, q, D, h_q, int64_t(rank_count) * pl->M, 128)) return st;
   if (zz_status_t st = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return st;
   if (zz_status_t st = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return st;
-  const bool pair = use_pair_kernel(D, group);
+  const bool pair = kc != kSingleCta;
   if (!pair)
     if (zz_status_t e = ensure_smem_attr<D>()) return e;
   void* base = nullptr;
@@ -1231,6 +1284,7 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = 1000000000ull;
   p.causal = 1;
+  p.pair_rows = kc == kPairRows ? 1 : 0;
   p.n_items = int(n_items);
   p.chunk_items = chunk_items_for(p.groups_per_kv);
   if (pair)

@@ -28,7 +28,8 @@ struct HalfDesc {
 };
 
 // One unit of attention work: rows [tile*128, tile*128+128) of a half, or for
-// pair lists the two tiles 2*tile and 2*tile+1.
+// pair lists the two tiles 2*tile and 2*tile+1, or for quad lists the four
+// tiles 4*tile .. 4*tile+3.
 struct WorkItem {
   int32_t half_id;
   int32_t tile;
@@ -39,7 +40,8 @@ constexpr int kStatusTimeout = 1;   // a bounded wait gave up
 constexpr int kStatusBadPage = 4;   // a page_table entry pointed outside the pool
 
 struct Workspace {  // byte offsets into the device workspace
-  size_t src_row, rank_tok, halves, tiles_all, tiles_rank, pairs_all, pairs_rank, status, total;
+  size_t src_row, rank_tok, halves, tiles_all, tiles_rank, pairs_all, pairs_rank, quads_all, quads_rank,
+      status, total;
 };
 
 }  // namespace zz
@@ -60,8 +62,8 @@ struct zz_plan {
   int64_t causal_pairs = 0;
   // device tables, host copies
   std::vector<zz::HalfDesc> halves;                               // [c*2*bs]
-  std::vector<zz::WorkItem> tiles_all, tiles_rank, pairs_all, pairs_rank;
-  std::vector<int32_t> tile_rank_off, pair_rank_off;              // [c+1]
+  std::vector<zz::WorkItem> tiles_all, tiles_rank, pairs_all, pairs_rank, quads_all, quads_rank;
+  std::vector<int32_t> tile_rank_off, pair_rank_off, quad_rank_off;   // [c+1]
   zz::Workspace ws{};
   void* dev_ws = nullptr;
   void* staging = nullptr;   // pinned host image of the workspace, made at the first upload

@@ -77,7 +77,7 @@ static void build_tables(zz_plan* p) {
     const int64_t last_key = int64_t(d.kv_pos0) + last_row;  // inclusive
     return last_key / zz::kTileN + 1;
   };
-  std::vector<Costed> tiles, pairs;
+  std::vector<Costed> tiles, pairs, quads;
   for (size_t id = 0; id < p->halves.size(); ++id) {
     const HalfDesc& d = p->halves[id];
     const int nt = (d.lq + zz::kTileM - 1) / zz::kTileM;
@@ -91,6 +91,12 @@ static void build_tables(zz_plan* p) {
       const int64_t cost = kv_tiles_upto_row(d, last) +
                            (2 * k + 1 < nt ? kv_tiles_upto_row(d, first_last) : 0);
       pairs.push_back({{int32_t(id), k}, d.rank, cost});
+    }
+    // Quads (CTA pairs, two row tiles per CTA): every tile of the quad runs to
+    // the keys of its last valid row tile.
+    for (int k = 0; 4 * k < nt; ++k) {
+      const int64_t last = std::min<int64_t>(int64_t(4 * k + 4) * zz::kTileM, d.lq) - 1;
+      quads.push_back({{int32_t(id), k}, d.rank, 4 * kv_tiles_upto_row(d, last)});
     }
   }
   auto by_cost = [](const Costed& a, const Costed& b) { return a.cost > b.cost; };
@@ -113,6 +119,8 @@ static void build_tables(zz_plan* p) {
   emit(tiles, true, p->tiles_rank, &p->tile_rank_off);
   emit(pairs, false, p->pairs_all, nullptr);
   emit(pairs, true, p->pairs_rank, &p->pair_rank_off);
+  emit(quads, false, p->quads_all, nullptr);
+  emit(quads, true, p->quads_rank, &p->quad_rank_off);
   // ---- workspace layout ----
   zz::Workspace& w = p->ws;
   size_t at = 0;
@@ -123,6 +131,8 @@ static void build_tables(zz_plan* p) {
   w.tiles_rank = at; at = align256(at + sizeof(WorkItem) * p->tiles_rank.size());
   w.pairs_all = at;  at = align256(at + sizeof(WorkItem) * p->pairs_all.size());
   w.pairs_rank = at; at = align256(at + sizeof(WorkItem) * p->pairs_rank.size());
+  w.quads_all = at;  at = align256(at + sizeof(WorkItem) * p->quads_all.size());
+  w.quads_rank = at; at = align256(at + sizeof(WorkItem) * p->quads_rank.size());
   w.status = at;     at = align256(at + 4 * sizeof(int32_t));
   w.total = at;
 }
@@ -354,6 +364,8 @@ extern "C" zz_status_t zz_plan_upload(zz_plan_t* p, void* dev, size_t bytes, voi
         {p->ws.tiles_rank, p->tiles_rank.data(), p->tiles_rank.size() * sizeof(zz::WorkItem)},
         {p->ws.pairs_all, p->pairs_all.data(), p->pairs_all.size() * sizeof(zz::WorkItem)},
         {p->ws.pairs_rank, p->pairs_rank.data(), p->pairs_rank.size() * sizeof(zz::WorkItem)},
+        {p->ws.quads_all, p->quads_all.data(), p->quads_all.size() * sizeof(zz::WorkItem)},
+        {p->ws.quads_rank, p->quads_rank.data(), p->quads_rank.size() * sizeof(zz::WorkItem)},
     };
     for (auto& part : parts)
       if (part.n) std::memcpy(img + part.off, part.src, part.n);

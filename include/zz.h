@@ -294,10 +294,10 @@ zz_status_t zz_ipc_close(void* base);
  * num_kv_heads"), null or misaligned pointers, rank range outside [0,c);
  * ZZ_ERR_UNSUPPORTED for d not in {64,128}, or for bf16 a page_size that is
  * neither 8, 16, 32, 64 nor a multiple of 128.
- * bf16 runs the tcgen05/TMEM/TMA kernel (fp32 accumulate and softmax); for
- * d = 128 with h_q/h_kv a multiple of 4 it runs on pairs of CTAs (clusters of
- * two that share each MMA; each CTA loads half of every K and V tile), else on
- * single CTAs.  fp32 runs a CUDA-core kernel in full fp32.
+ * bf16 runs the tcgen05/TMEM/TMA kernel (fp32 accumulate and softmax): for
+ * d = 128 on pairs of CTAs (clusters of two that share each MMA; each CTA
+ * loads half of every K and V tile), for d = 64 on single CTAs.  fp32 runs a
+ * CUDA-core kernel in full fp32.
  */
 zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_count,
                             const void* q, const void* k_pool, const void* v_pool,

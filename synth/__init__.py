@@ -11,7 +11,10 @@ Recipe (all seeded):
     natural token order, standard normal times ``scale``; bf16 tensors are the
     fp32 draw rounded to nearest-even;
   * pool pages: a seeded permutation of the pool's pages, handed out to the
-    sequences in order, each sequence starting on a page boundary.
+    sequences in order, each sequence starting on a page boundary;
+  * growing scores (optional): key row at position t of its sequence scaled by
+    ``1 + per_tile * t / 128``, so that attention scores grow along the
+    sequence (drives the kernel's redo of tiles whose row sum leaves range).
 """
 from __future__ import annotations
 
@@ -64,6 +67,15 @@ def qkv(total_tokens: int, h_q: int, h_kv: int, d: int, seed: int, scale: float,
     k = normal((total_tokens, h_kv, d), seed, scale, dtype, device, g)
     v = normal((total_tokens, h_kv, d), seed, scale, dtype, device, g)
     return q, k, v
+
+
+def key_ramp(k: torch.Tensor, seq_lens, per_tile: float) -> torch.Tensor:
+    """``k`` ``[T, H, D]`` (natural order, sequences back to back) with the row at
+    position t of its sequence scaled by ``1 + per_tile * t / 128`` (in fp32,
+    then cast back to ``k``'s dtype)."""
+    pos = torch.cat([torch.arange(n, dtype=torch.float32) for n in seq_lens]).to(k.device)
+    f = (1.0 + per_tile * pos / 128.0).view(-1, 1, 1)
+    return (k.float() * f).to(k.dtype)
 
 
 @dataclass

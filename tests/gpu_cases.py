@@ -39,6 +39,7 @@ class Case:
     page_seed: int | None = 1
     prefix: list | None = None   # cached-prefix tokens per sequence (already in the pool)
     causal: bool = True
+    k_ramp: float = 0.0          # > 0: key magnitudes grow along each sequence (synth.key_ramp)
 
 
 class Run:
@@ -57,6 +58,8 @@ class Run:
         gdev = gen_device or ("cpu" if T * c.h_q * c.d < 2**27 else device)
         # natural-order inputs: prefix tokens first, then the extend tokens, per sequence
         self.q, k_all, v_all = synth.qkv(sum(full), c.h_q, c.h_kv, c.d, c.seed, c.scale, c.dtype, gdev)
+        if c.k_ramp:
+            k_all = synth.key_ramp(k_all, full, c.k_ramp)
         starts = np.cumsum([0] + full)
         ext_rows = np.concatenate([np.arange(starts[s] + prefix[s], starts[s + 1]) for s in range(len(full))])
         ext_idx = torch.from_numpy(ext_rows).to(gdev)

@@ -61,6 +61,37 @@ def test_small_cases_every_row(case):
     _check_full(Run(case))
 
 
+# Key magnitudes that grow along the sequence: later tiles' scores exceed the
+# first tile's maximum by far more than the kernel's range for a kept tile, so
+# the kernel must redo tiles (new maximum, O and l rescaled) several times per
+# row, in every kernel and mode.
+REDO = [
+    Case(4, [1500, 700], 8, 2, 128, page_size=16, k_ramp=4.0),                   # CTA pairs, heads
+    Case(2, [2100], 4, 4, 128, page_size=64, k_ramp=4.0),                        # CTA pairs, row tiles
+    Case(2, [1300], 4, 2, 64, page_size=32, k_ramp=4.0),                         # single CTA, head_dim 64
+    Case(2, [900], 4, 2, 128, page_size=16, k_ramp=8.0, causal=False),           # non-causal
+    Case(2, [700, 300], 4, 2, 128, page_size=16, prefix=[300, 64], k_ramp=8.0),  # cached prefix
+]
+
+
+def _max_growth_log2(run: Run) -> float:
+    """Largest rise of a 128-key tile's score maximum (log2 units) over the first
+    tile's, for the last query row of sequence 0, head 0."""
+    c = run.case
+    k = run.k_seqs[0][:, 0].double().cpu().numpy()
+    q = run.q[c.lens[0] - 1, 0].double().cpu().numpy()
+    s = (k @ q) * run.softmax_scale / np.log(2.0)
+    tiles = [s[i:i + 128].max() for i in range(0, len(s), 128)]
+    return float(max(tiles) - tiles[0])
+
+
+@pytest.mark.parametrize("case", REDO, ids=["pair-heads", "pair-rows", "single-d64", "noncausal", "prefix"])
+def test_growing_scores_redo_tiles_every_row(case):
+    run = Run(case)
+    assert _max_growth_log2(run) > 24.0      # a row sum of at least 2^24 > 2^16: redone
+    _check_full(run)
+
+
 def test_c4_L4096_gqa8_every_row():
     _check_full(Run(Case(4, [4096], 32, 4, 128, page_size=16)))
 

@@ -18,8 +18,8 @@
 //   warp  8    MMA issue (one thread) + TMEM allocation
 //   warp  9    TMA producer: Q once, then K/V stages (V_{j-1}, K_j) into a smem ring
 //   warps 10-11 idle
-// Launched at 168 registers a thread; the softmax warpgroups grow to 216 and
-// the third warpgroup shrinks to 72 (216 + 216 + 72 = 3 x 168 per SM
+// Launched at 168 registers a thread; the softmax warpgroups grow to 192 and
+// the third warpgroup shrinks to 120 (192 + 192 + 120 = 3 x 168 per SM
 // sub-partition), so a whole 128-column row of S stays in registers with no
 // spills.
 // TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [256+D,256+2D).
@@ -27,9 +27,11 @@
 // feeds the P.V MMA straight from TMEM.  The MMA order per K/V tile j is
 //   PV0(j)  S0(j+1)  PV1(j)  S1(j+1)
 // so each softmax group works on one tile while the tensor core runs the
-// other group's MMAs.  The softmax keeps a running maximum in log2 units and
-// only rescales O (in TMEM) when the maximum grows by more than 8, so most
-// tiles skip the correction.  Tiles past the causal diagonal are never loaded.
+// other group's MMAs.  The softmax takes the exact row maximum on a row's
+// first tile only and afterwards exponentiates against the running maximum,
+// redoing a tile (with O rescaled in TMEM) only when its row sum leaves the
+// range (softmax_tile), so the row-maximum pass is off the per-tile chain.
+// Tiles past the causal diagonal are never loaded.
 //
 // attn_fwd_pair (further down) is the same pipeline on clusters of two CTAs
 // whose MMAs are shared (tcgen05 .cta_group::2, M = 256), for head_dim 128:
@@ -65,11 +67,17 @@ namespace {
 using namespace zz::dev;
 
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 216, kRegsOther = 72;
+constexpr uint32_t kRegsSoftmax = 192, kRegsOther = 120;
 constexpr int kWarpMma = 8;
 constexpr int kWarpLoad = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 256 between rescales
+// Online softmax with a lagging maximum: the row maximum is taken exactly on a
+// row's first K/V tile only.  Later tiles use the running maximum m as it is;
+// any m at or below the true running maximum gives the same O and l (both
+// carry the factor 2^-m), it only has to keep P finite.  The tile's row sum
+// bounds every P of the tile, so a tile whose sum exceeds kRedoSum is redone
+// against its own maximum after O and l are rescaled.
+constexpr float kRedoSum = 65536.0f;   // P <= 2^16 on every tile that is kept
 // Bit e of kPolyMask: exponential pair e (of the 16 pairs of each 32-column
 // chunk of an S row) is evaluated with the FMA-pipe polynomial of exp2_poly.h
 // instead of MUFU ex2, on tiles that need no causal mask (masked tiles keep
@@ -145,6 +153,82 @@ __device__ __forceinline__ int tiles_for(const HalfDesc& h, int q0, int causal) 
   if (!causal) return (h.kv_full + 127) / 128;
   const int last_row = min(q0 + 128, h.lq) - 1;
   return (h.kv_pos0 + last_row) / 128 + 1;
+}
+
+// Softmax of one K/V tile for one query row (thread = TMEM lane): S(j) of the
+// row in registers (causal mask applied) -> P = 2^(s*scale*log2e - m) as bf16
+// pairs over the first 64 columns of the row's S in TMEM; updates m and l and,
+// when a tile is redone, rescales the row's O (D columns at t_o) in TMEM.
+// S(j) completing implies P.V(j-1) completed, so O is stable here.  All TMEM
+// accesses are warp-wide (.sync.aligned), so every branch around them is
+// taken by the whole warp.
+template <int D>
+__device__ __forceinline__ void softmax_tile(const uint32_t (&sr)[128], int j, bool masked, float scale_log2,
+                                             uint32_t t_s, uint32_t t_o, float& m, float& l) {
+  auto row_max = [&]() {   // 8 independent max3 chains (short dependency depth)
+    float pm[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) pm[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
+#pragma unroll
+    for (int c = 16; c < 128; c += 16)
+#pragma unroll
+      for (int q = 0; q < 8; q += 2)
+        pm[q] = fmax3(pm[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + q + 8])),
+        pm[q + 1] = fmax3(pm[q + 1], __uint_as_float(sr[c + q + 1]), __uint_as_float(sr[c + q + 9]));
+    return fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], fmax3(pm[5], pm[6], pm[7]))) * scale_log2;
+  };
+  // P of the whole row: packed FMA, ex2 (or the polynomial), packed running
+  // sum, bf16 pairs into TMEM.  Returns the tile's row sum.
+  auto exp_pass = [&](auto use_poly) {
+    const float2 sl2 = make_float2(scale_log2, scale_log2);
+    const float2 nm2 = make_float2(-m, -m);
+    float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int col = c * 32 + 2 * e;
+        float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2, nm2);
+        if (decltype(use_poly)::value && ((kPolyMask >> e) & 1u)) {
+          x = exp2_poly2(x);
+        } else {
+          x.x = ex2(x.x);
+          x.y = ex2(x.y);
+        }
+        acc4[e & 3] = fadd2(acc4[e & 3], x);
+        pk[e] = pack_bf16x2(x.x, x.y);
+      }
+      tmem_st16(t_s + c * 16, pk);
+    }
+    const float2 acc = fadd2(fadd2(acc4[0], acc4[1]), fadd2(acc4[2], acc4[3]));
+    return acc.x + acc.y;
+  };
+  auto exp_any = [&]() {
+    return (kPolyMask == 0u || masked) ? exp_pass(std::false_type{}) : exp_pass(std::true_type{});
+  };
+  if (j == 0) m = row_max();
+  float l_tile = exp_any();
+  if (j > 0 && __any_sync(0xffffffffu, !(l_tile <= kRedoSum))) {
+    // Rows whose maximum did not move keep m (factor exactly 1, same P).
+    const float m_new = fmaxf(m, row_max());
+    const float f = ex2(m - m_new);
+    m = m_new;
+    tmem_wait_st();                      // the first pass's P lands before it is overwritten
+    l_tile = exp_any();
+    l *= f;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(t_o + c * 32, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+      tmem_st32(t_o + c * 32, o);
+    }
+  }
+  l += l_tile;
 }
 
 template <int D>
@@ -373,14 +457,14 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int slot = t % C::kStages;
         if (!(ok = wait_parity(&bars->kv_full[slot], uint32_t(t / C::kStages) & 1u, abort, p.timeout_ns))) break;
         if (j < n0) {
-          if (!(ok = wait_parity(&bars->p_full[0], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+          if (!(ok = wait_spin(&bars->p_full[0], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
           tc_fence_after();
           issue_pv(C::kColO0, C::kColS0, slot, j > 0);
           if (j == n0 - 1) mma_commit(&bars->o_full[0]);
           else { issue_s(C::kColS0, dq0, slot); mma_commit(&bars->s_full[0]); }
         }
         if (j < n1) {
-          if (!(ok = wait_parity(&bars->p_full[1], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+          if (!(ok = wait_spin(&bars->p_full[1], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
           tc_fence_after();
           issue_pv(C::kColO1, C::kColS1, slot, j > 0);
           if (j == n1 - 1) mma_commit(&bars->o_full[1]);
@@ -428,73 +512,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int c = 0; c < 128; ++c)
           if (c >= limit) sr[c] = 0xFF800000u;     // -inf
       }
-      // Row maximum as 8 independent max3 chains (short dependency depth).
-      float pm[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) pm[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
-#pragma unroll
-      for (int c = 16; c < 128; c += 16)
-#pragma unroll
-        for (int q = 0; q < 8; q += 2)
-          pm[q] = fmax3(pm[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + q + 8])),
-          pm[q + 1] = fmax3(pm[q + 1], __uint_as_float(sr[c + q + 1]), __uint_as_float(sr[c + q + 9]));
-      const float mx = fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], fmax3(pm[5], pm[6], pm[7])));
-      const float m_tile = mx * p.scale_log2;
-      if (j == 0) {
-        m = m_tile;
-      } else {
-        // Rescale when the maximum grows by more than the threshold.  The TMEM
-        // loads and stores are warp-wide, so the whole warp takes the branch
-        // when any of its rows needs it; rows that keep their maximum use a
-        // factor of exactly 1.  S(j) completing implies P.V(j-1) completed:
-        // O is stable here.
-        const bool need = m_tile > m + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = need ? m_tile : m;
-          const float f = ex2(m - m_new);
-          l *= f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_o + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(t_o + c * 32, o);
-          }
-          m = m_new;
-        }
-      }
-      // P = 2^(s*scale*log2e - m): packed FMA, ex2 (or the polynomial), packed
-      // running sum, bf16 pairs written over the first 64 columns of S.
-      const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
-      const float2 nm2 = make_float2(-m, -m);
-      float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
-      auto exp_row = [&](auto use_poly) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int col = c * 32 + 2 * e;
-            float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2, nm2);
-            if (decltype(use_poly)::value && ((kPolyMask >> e) & 1u)) {
-              x = exp2_poly2(x);
-            } else {
-              x.x = ex2(x.x);
-              x.y = ex2(x.y);
-            }
-            acc4[e & 3] = fadd2(acc4[e & 3], x);
-            pk[e] = pack_bf16x2(x.x, x.y);
-          }
-          tmem_st16(t_s + c * 16, pk);
-        }
-      };
-      if (kPolyMask == 0u || masked) exp_row(std::false_type{});
-      else exp_row(std::true_type{});
-      const float2 acc = fadd2(fadd2(acc4[0], acc4[1]), fadd2(acc4[2], acc4[3]));
-      l += acc.x + acc.y;
+      softmax_tile<D>(sr, j, masked, p.scale_log2, t_s, t_o, m, l);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[g]);
@@ -566,7 +584,7 @@ struct PairCfg {
 };
 static_assert(PairCfg::kSmem <= 232448, "227 KB of shared memory per CTA");
 // setmaxnreg split of the pair kernel (the one without spills for its code).
-constexpr uint32_t kPairRegsSoftmax = 208, kPairRegsOther = 88;
+constexpr uint32_t kPairRegsSoftmax = 192, kPairRegsOther = 120;
 static_assert(2 * kPairRegsSoftmax + kPairRegsOther <= 3 * 168, "register split exceeds the launch's registers");
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -815,12 +833,12 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int t = j + 1;                    // stage with V_j and K_{j+1}
         const int slot = t % C::kStages;
         if (!(ok = wait_parity(&bars->kv_full[slot], uint32_t(t / C::kStages) & 1u, abort, p.timeout_ns))) break;
-        if (!(ok = wait_parity(&bars->p_full[0], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+        if (!(ok = wait_spin(&bars->p_full[0], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
         tc_fence_after();
         issue_pv(C::kColO0, C::kColS0, slot, j > 0);
         if (j == n - 1) mma_commit_pair(&bars->o_full[0], both);
         else { issue_s(C::kColS0, dq0, slot); mma_commit_pair(&bars->s_full[0], both); }
-        if (!(ok = wait_parity(&bars->p_full[1], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
+        if (!(ok = wait_spin(&bars->p_full[1], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
         tc_fence_after();
         issue_pv(C::kColO1, C::kColS1, slot, j > 0);
         if (j == n - 1) mma_commit_pair(&bars->o_full[1], both);
@@ -863,62 +881,7 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int c = 0; c < 128; ++c)
           if (c >= limit) sr[c] = 0xFF800000u;
       }
-      float pm[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) pm[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
-#pragma unroll
-      for (int c = 16; c < 128; c += 16)
-#pragma unroll
-        for (int q = 0; q < 8; q += 2)
-          pm[q] = fmax3(pm[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + q + 8])),
-          pm[q + 1] = fmax3(pm[q + 1], __uint_as_float(sr[c + q + 1]), __uint_as_float(sr[c + q + 9]));
-      const float mx = fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], fmax3(pm[5], pm[6], pm[7])));
-      const float m_tile = mx * p.scale_log2;
-      if (j == 0) {
-        m = m_tile;
-      } else {
-        // Rescale when the maximum grows by more than the threshold.  The TMEM
-        // loads and stores are warp-wide, so the whole warp takes the branch
-        // when any of its rows needs it; rows that keep their maximum use a
-        // factor of exactly 1.  S(j) completing implies P.V(j-1) completed:
-        // O is stable here.
-        const bool need = m_tile > m + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = need ? m_tile : m;
-          const float f = ex2(m - m_new);
-          l *= f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_o + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(t_o + c * 32, o);
-          }
-          m = m_new;
-        }
-      }
-      const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
-      const float2 nm2 = make_float2(-m, -m);
-      float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int col = c * 32 + 2 * e;
-          float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2, nm2);
-          x.x = ex2(x.x);
-          x.y = ex2(x.y);
-          acc4[e & 3] = fadd2(acc4[e & 3], x);
-          pk[e] = pack_bf16x2(x.x, x.y);
-        }
-        tmem_st16(t_s + c * 16, pk);
-      }
-      const float2 acc = fadd2(fadd2(acc4[0], acc4[1]), fadd2(acc4[2], acc4[3]));
-      l += acc.x + acc.y;
+      softmax_tile<D>(sr, j, masked, p.scale_log2, t_s, t_o, m, l);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_cluster(p_full_lead);         // the leader's barrier, from either CTA

@@ -69,6 +69,39 @@ __device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity, vola
   }
 }
 
+// Non-blocking probe of the same phase (mbarrier.test_wait never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// wait_parity for a thread with nothing else to do (the MMA issuer): polls
+// with test_wait instead of suspending in try_wait, which wakes it sooner
+// after the phase completes.  Same bounds: the abort flag and the timeout are
+// checked every 64 polls.
+__device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t timeout_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > timeout_ns) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // Drain wait used on the way out: ignores the abort flag (in-flight copies
 // and MMAs must land before the CTA releases shared memory and TMEM) but is
 // still bounded by `timeout_ns`.

@@ -305,6 +305,53 @@ def oracle_sample(cp, lens, h_q, h_kv, d, budget_s: float, k_seqs=None, v_seqs=N
     return flops, time.perf_counter() - t0, rows
 
 
+def oracle_config_timing(cp, lens, h_q, h_kv, d, full_budget_s: float = 12.0, sample_s: float = 1.5, seed=7):
+    """The oracle on one configuration's shape, on the host cores: plan build and
+    K+V rerange in full; attention in full when its FLOPs fit ``full_budget_s``
+    at the oracle's measured rate, else on sampled query rows for ``sample_s``
+    (labelled as sampled).  Inputs are seeded CPU draws of the same shapes."""
+    import synth
+    from oracle import attention as OA
+    from oracle import plan as OP
+    from oracle import rerange as OR
+    T = sum(lens)
+    t0 = time.perf_counter()
+    ref = OP.build_metadata(cp, T, extend_lens=lens)
+    plan_ms = (time.perf_counter() - t0) * 1e3
+    pool = synth.paged_pool(lens, 16, seed=1)
+    g = np.random.default_rng(seed)
+    kv = [g.integers(-32768, 32767, size=(cp * ref.M, h_kv, d), dtype=np.int16) for _ in range(2)]
+    empty = np.zeros((pool.num_slots, h_kv, d), np.int16)
+    t0 = time.perf_counter()
+    for x in kv:
+        OR.rerange_to_pool(x, ref, empty, pool.out_cache_loc)
+    rr_s = time.perf_counter() - t0
+    del kv, empty
+    out = {"plan_ms": plan_ms, "rerange_gbs": 2 * 2 * T * h_kv * d * 2 / rr_s / 1e9, "cores_rerange": 1}
+    # attention: a short sample gives the rate; the full run only when it fits the budget
+    f, t, rows = oracle_sample(cp, lens, h_q, h_kv, d, sample_s, seed=seed)
+    rate = f / t
+    total = OA.plan_flops(ref, h_q, d)
+    if total / rate <= full_budget_s:
+        starts = np.cumsum([0] + lens)
+        q_all = synth.normal((T, h_q, d), seed, 0.5, "bf16", "cpu", g).double().numpy()
+        k_all = synth.normal((T, h_kv, d), seed, 0.5, "bf16", "cpu", g).double().numpy()
+        v_all = synth.normal((T, h_kv, d), seed, 0.5, "bf16", "cpu", g).double().numpy()
+        ks = [k_all[starts[i]:starts[i + 1]] for i in range(len(lens))]
+        vs = [v_all[starts[i]:starts[i + 1]] for i in range(len(lens))]
+        t0 = time.perf_counter()
+        for r in range(cp):
+            OA.run_rank(ref, r, OR.shard(q_all, ref, r), ks, vs, 1.0 / math.sqrt(d))
+        t = time.perf_counter() - t0
+        out.update(attn_tflops=total / t / 1e12, attn_sample=f"full ({total / 1e9:.2f} GFLOP in {t:.2f} s)")
+    else:
+        out.update(attn_tflops=rate / 1e12,
+                   attn_sample=f"sampled: {rows} query rows x {h_q} heads over every rank/half, {t:.1f} s")
+    out["cores_attention"] = blas_threads()
+    out["kind"] = "oracle"
+    return out
+
+
 # ----------------------------------------------------------------- reference arm
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -578,7 +625,7 @@ def main_gpu(args):
     if world == 1 and not args.no_per_config:
         del q_mine, out, k_local, v_local, k_g, v_g, k_pool, v_pool
         torch.cuda.empty_cache()
-        per_config = per_config_attention(torch, zz, synth, dev)
+        per_config = per_config_attention(torch, zz, synth, dev, with_oracle=not args.no_cpu_baseline)
 
     peaks, peaks_src = load_peaks()
     peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
@@ -666,7 +713,7 @@ PER_CONFIG = [
      for hq, hkv in ((32, 32), (32, 8), (32, 1)) for cp in (2, 4, 8)]
 
 
-def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 512):
+def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 512, with_oracle: bool = True):
     """Attention (and rerange) kernel time on every configuration's shape.
 
     Per configuration: seeded inputs, plan, shard, rerange into the paged pool,
@@ -733,6 +780,8 @@ def per_config_attention(torch, zz, synth, dev, reps: int = 7, flush_mb: int = 5
             row["attn_frac_of_bf16_sustained"] = tf / sus
         else:
             row["attn_kernel"] = "fp32 CUDA-core kernel (no tensor-core peak applies)"
+        if with_oracle:
+            row["cpu_baseline"] = oracle_config_timing(cp, lens, h_q, h_kv, d)
         out_rows.append(row)
         del q, kg, vg, kp, vp, out, page_table, loc, plan
         torch.cuda.empty_cache()

@@ -30,6 +30,16 @@ def _free_port():
         return s.getsockname()[1]
 
 
+def _put_and_exit(q, item, code):
+    """Queue ``item`` and leave at once.  ``put`` only hands the item to a feeder
+    thread; close + join_thread flush it to the pipe before os._exit, which
+    would otherwise drop it."""
+    q.put(item)
+    q.close()
+    q.join_thread()
+    os._exit(code)
+
+
 def _init(rank, world, port, timeout_s=60):
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -149,8 +159,7 @@ def _fail_worker(rank, world, port, mode, out_q):
         out_q.put((rank, "completed", 0.0))
     except RuntimeError as e:
         if "injected" in str(e):
-            out_q.put((rank, "raised", 0.0))
-            os._exit(1)
+            _put_and_exit(out_q, (rank, "raised", 0.0), 1)
         raise
 
 
@@ -184,15 +193,14 @@ def _collective_worker(rank, world, port, out_q):
     t = torch.ones(1)
     if rank == 1:
         time.sleep(6)                                # never joins the collective in time
-        out_q.put((rank, "slept", 0.0))
-        os._exit(0)
+        _put_and_exit(out_q, (rank, "slept", 0.0), 0)
     t0 = time.monotonic()
     try:
         dist.all_reduce(t)
-        out_q.put((rank, "returned", time.monotonic() - t0))
+        item = (rank, "returned", time.monotonic() - t0)
     except Exception as e:  # gloo raises on the process-group timeout
-        out_q.put((rank, type(e).__name__, time.monotonic() - t0))
-    os._exit(0)
+        item = (rank, type(e).__name__, time.monotonic() - t0)
+    _put_and_exit(out_q, item, 0)
 
 
 def test_a_collective_nobody_joins_ends_with_an_error_within_the_group_timeout():

@@ -668,7 +668,7 @@ def main_gpu(args):
                      "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel runs inside a long step)",
                      "traffic": traffic},
         "e2e": e2e,
-        "gpu_launches": (1 + (r_per if push else 1)) * args.steps,
+        "gpu_launches": (2 + (r_per if push else 1)) * args.steps,   # plan upload, rerange (or pushes), attention
         "device_status": status,
         "clocks": clocks,
         "cpu_baseline": cpu,

@@ -118,9 +118,11 @@ size_t zz_plan_workspace_bytes(const zz_plan_t* plan);
  * and remember that address for later calls.  The plan must outlive the copy.
  * The first upload of a plan lays its tables out in pinned host memory owned
  * by the plan (cudaMallocHost, freed by zz_plan_destroy; make that first call
- * outside stream capture).  Every upload is then one asynchronous copy from
- * there, which neither waits for `stream` nor blocks the calling thread, and
- * also clears the status word.
+ * outside stream capture).  Every upload is then one small kernel on `stream`
+ * that reads that image through its device mapping: it does not block the
+ * calling thread, and unlike a copy-engine transfer it does not queue behind
+ * other streams' host<->device copies (e.g. the next batch's inputs).  The
+ * upload also clears the status word.
  */
 zz_status_t zz_plan_upload(zz_plan_t* plan, void* dev_workspace, size_t bytes, void* stream);
 

@@ -67,6 +67,7 @@ struct zz_plan {
   zz::Workspace ws{};
   void* dev_ws = nullptr;
   void* staging = nullptr;   // pinned host image of the workspace, made at the first upload
+  void* staging_dev = nullptr;   // the same image as the device sees it (mapped pinned memory)
   // Device ordinal of the last zz_attn_prefill_noalloc call made with this plan
   // (-1: none); zz_plan_device_status then also reads the static status word.
   mutable std::atomic<int> noalloc_dev{-1};

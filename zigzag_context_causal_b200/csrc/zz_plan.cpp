@@ -338,6 +338,18 @@ extern "C" zz_status_t zz_plan_get(const zz_plan_t* p, int rank, zz_field_t fiel
 
 extern "C" size_t zz_plan_workspace_bytes(const zz_plan_t* p) { return p ? p->ws.total : 0; }
 
+namespace {
+// The upload itself: plain 16-byte loads from the pinned (device-mapped) host
+// image, one kernel on the caller's stream.  A copy-engine transfer
+// (cudaMemcpyAsync) would queue behind other streams' host<->device copies,
+// e.g. the next batch's inputs, and stall the stream for as long as they take.
+__global__ void __launch_bounds__(256) upload_tables(const int4* __restrict__ src, int4* __restrict__ dst,
+                                                     size_t n16) {
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += size_t(gridDim.x) * blockDim.x)
+    dst[i] = src[i];
+}
+}  // namespace
+
 extern "C" zz_status_t zz_plan_upload(zz_plan_t* p, void* dev, size_t bytes, void* stream) {
   ZZ_NVTX("zz_plan_upload");
   if (!p || !dev) return zz::fail(ZZ_ERR_INVALID_ARG, "zz_plan_upload: NULL argument");
@@ -347,8 +359,8 @@ extern "C" zz_status_t zz_plan_upload(zz_plan_t* p, void* dev, size_t bytes, voi
   auto s = static_cast<cudaStream_t>(stream);
   // The tables never change after zz_plan_create: lay them out once in pinned
   // host memory exactly as in the workspace (status word zero), so that every
-  // upload is one asynchronous copy that neither waits for the stream nor
-  // blocks the calling thread.
+  // upload is one kernel that reads that image over the bus: it neither blocks
+  // the calling thread nor waits for other streams' copies.
   if (!p->staging) {
     void* h = nullptr;
     cudaError_t e = cudaMallocHost(&h, p->ws.total);
@@ -369,9 +381,20 @@ extern "C" zz_status_t zz_plan_upload(zz_plan_t* p, void* dev, size_t bytes, voi
     };
     for (auto& part : parts)
       if (part.n) std::memcpy(img + part.off, part.src, part.n);
+    void* mapped = nullptr;
+    e = cudaHostGetDevicePointer(&mapped, h, 0);
+    if (e != cudaSuccess) {
+      cudaFreeHost(h);
+      return zz::fail(ZZ_ERR_CUDA, std::string("zz_plan_upload: mapping the staging: ") + cudaGetErrorString(e));
+    }
     p->staging = h;
+    p->staging_dev = mapped;
   }
-  cudaError_t e = cudaMemcpyAsync(dev, p->staging, p->ws.total, cudaMemcpyHostToDevice, s);
+  const size_t n16 = p->ws.total / 16;   // the workspace size is a multiple of 256 bytes
+  const size_t blocks = std::min<size_t>((n16 + 255) / 256, 1024);
+  upload_tables<<<unsigned(blocks), 256, 0, s>>>(static_cast<const int4*>(p->staging_dev), static_cast<int4*>(dev),
+                                                 n16);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return zz::fail(ZZ_ERR_CUDA, std::string("zz_plan_upload: ") + cudaGetErrorString(e));
   p->dev_ws = dev;

@@ -1129,17 +1129,21 @@ zz_status_t launch_bf16(const zz_plan_t* pl, int rank_begin, int rank_count, con
       return e;
     return enqueue_pair(pq, pk, pv, grid, p, stream);
   }
-  if (zz_status_t e = get_encoder()) return e;
-  CUtensorMap tq, tk, tv;
-  if (zz_status_t e = encode_3d(&tq, q, D, h_q, q_rows, 128)) return e;
-  if (zz_status_t e = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return e;
-  if (zz_status_t e = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return e;
-  p.chunk_items = chunk_items_for(p.groups_per_kv);
-  if (zz_status_t e = ensure_smem_attr<D>()) return e;
-  attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));
-  return ZZ_OK;
+  if constexpr (D == 128) {
+    return fail(ZZ_ERR_UNSUPPORTED, "head_dim 128 runs on the CTA-pair kernel only");   // kernel_for never gets here
+  } else {
+    if (zz_status_t e = get_encoder()) return e;
+    CUtensorMap tq, tk, tv;
+    if (zz_status_t e = encode_3d(&tq, q, D, h_q, q_rows, 128)) return e;
+    if (zz_status_t e = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return e;
+    if (zz_status_t e = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return e;
+    p.chunk_items = chunk_items_for(p.groups_per_kv);
+    if (zz_status_t e = ensure_smem_attr<D>()) return e;
+    attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));
+    return ZZ_OK;
+  }
 }
 
 bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
@@ -1215,8 +1219,10 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   if (zz_status_t st = encode_3d(&tk, k_pool, D, h_kv, num_slots, box_rows)) return st;
   if (zz_status_t st = encode_3d(&tv, v_pool, D, h_kv, num_slots, box_rows)) return st;
   const bool pair = kc != kSingleCta;
-  if (!pair)
-    if (zz_status_t e = ensure_smem_attr<D>()) return e;
+  if constexpr (D != 128) {
+    if (!pair)
+      if (zz_status_t e = ensure_smem_attr<D>()) return e;
+  }
   void* base = nullptr;
   if (zz_status_t e = static_scratch_address(&base)) return e;
   int dev = 0;
@@ -1281,10 +1287,14 @@ zz_status_t launch_bf16_static(const zz_plan_t* pl, int rank_begin, int rank_cou
   }
   pl->noalloc_dev.store(dev);
   if (pair) return enqueue_pair(tq, tk, tv, grid, p, stream);
-  attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));
-  return ZZ_OK;
+  if constexpr (D == 128) {
+    return fail(ZZ_ERR_UNSUPPORTED, "head_dim 128 runs on the CTA-pair kernel only");   // kernel_for never gets here
+  } else {
+    attn_fwd_sm100<D><<<unsigned(grid), kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ZZ_ERR_CUDA, std::string("attn_fwd_sm100 launch: ") + cudaGetErrorString(e));
+    return ZZ_OK;
+  }
 }
 
 }  // namespace

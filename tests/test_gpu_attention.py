@@ -153,3 +153,38 @@ def test_L32768_head_ratio_sweep_every_tile(h_q, h_kv, cp):
 
 def test_long_context_c8_L131072_every_tile():
     _check_sampled(Run(Case(8, [131072], 64, 8, 128, page_size=64)))
+
+
+def _random_cases(n: int, seed: int = 2024):
+    """Seeded random small configurations: cp size, batch and ragged lengths,
+    GQA group (odd groups and MHA included), head_dim, page size, cached
+    prefix, causal or not, and growing scores; sized so that the oracle checks
+    every output row in about a second each."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        cp = int(rng.choice([2, 3, 4, 8]))
+        bs = int(rng.integers(1, 4))
+        lens = [int(x) for x in rng.integers(2 * cp, 900 // bs + 2 * cp, bs)]
+        h_kv = int(rng.choice([1, 2, 4]))
+        group = int(rng.choice([1, 2, 3, 4, 8]))
+        h_q = h_kv * group
+        if h_q > 16:
+            h_kv, h_q = 1, group
+        d = int(rng.choice([64, 128]))
+        ps = int(rng.choice([8, 16, 32, 64, 128, 256]))
+        prefix = [int(x) for x in rng.integers(0, 300, bs)] if rng.random() < 0.3 else None
+        causal = bool(rng.random() < 0.8)
+        ramp = 4.0 if rng.random() < 0.2 else 0.0
+        out.append(Case(cp, lens, h_q, h_kv, d, page_size=ps, prefix=prefix, causal=causal, k_ramp=ramp,
+                        seed=int(rng.integers(0, 1000))))
+    return out
+
+
+RANDOM = _random_cases(32)
+
+
+@pytest.mark.parametrize("case", RANDOM, ids=lambda c: f"c{c.cp}-L{c.lens}-{c.h_q}/{c.h_kv}-d{c.d}-ps{c.page_size}"
+                         f"{'-pre' if c.prefix else ''}{'' if c.causal else '-nc'}{'-ramp' if c.k_ramp else ''}")
+def test_random_small_configs_every_row(case):
+    _check_full(Run(case))

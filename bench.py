@@ -43,6 +43,7 @@ WORKLOADS = {
     "varlen": (4, "varlen", 32, 4, 128, 16,
                "c=4 varlen 8 seqs U[1000,8192] Hq/Hkv=32/4 D=128 bf16 page 16"),
     "mid": (8, [32768], 64, 8, 128, 64, "c=8 L=32768 Hq/Hkv=64/8 D=128 bf16 page 64"),
+    "sweep-gqa4": (8, [32768], 32, 8, 128, 16, "c=8 L=32768 Hq/Hkv=32/8 D=128 bf16 page 16"),
 }
 METRIC = "zigzag CP prefill attention TFLOP/s (% BF16 peak) + KV rerange GB/s (% HBM) on 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}

@@ -36,7 +36,11 @@
 // attn_fwd_pair (further down) is the same pipeline on clusters of two CTAs
 // whose MMAs are shared (tcgen05 .cta_group::2, M = 256), for head_dim 128:
 // per SM it loads half the K/V bytes and issues half the TMA boxes, which is
-// what bounds small pages.
+// what bounds small pages.  It is persistent: a cluster that finishes a work
+// unit takes the unit of a cluster that has not started yet, by cancelling
+// that cluster's launch (cluster launch control), so the next unit's Q load
+// and first S overlap the current unit's last P.V and epilogue and no
+// cluster pays the barrier/TMEM set-up twice.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -140,7 +144,50 @@ struct Bars {
   uint64_t kv_empty[8];
   uint32_t tmem_base;
   int abort;
+  // CTA-pair kernel: the ring that hands each cluster's next work unit to
+  // every role of both CTAs, and the cluster-launch-control response.
+  uint64_t unit_full[4];
+  uint64_t unit_empty[4];   // leader CTA only
+  uint64_t clc_full;
+  alignas(16) uint32_t clc_resp[4];
+  int unit_id[4];
+  uint32_t clc_issued;   // cancel requests issued (by the MMA thread)
 };
+
+// The unit ring: entry k (slot k % kUnitRing) holds the cluster's (k + 2)-th
+// work unit (the first is its own blockIdx), -1 once none is left.  The
+// leader's producer writes each entry into both CTAs; every other role of
+// both CTAs takes it and frees it with one arrival on the leader's unit_empty.
+constexpr int kUnitRing = 4;
+// The MMA thread asks for the next unit kClcLead K/V tiles before it issues
+// the unit's last S (that is, about kClcLead + 1 tiles before the cluster is
+// free): late enough that the hand-out stays dynamic, early enough that the
+// answer is there when the producer needs the next Q.
+constexpr int kClcLead = 2;
+constexpr int kUnitReaders = 18;   // leader: MMA thread + 8 softmax warps; peer: producer + 8 softmax warps
+
+__device__ __forceinline__ bool ring_put(Bars* bars, uint32_t k, int vc, volatile int* abort,
+                                         uint64_t timeout_ns) {
+  const int slot = int(k % kUnitRing);
+  const uint32_t use = k / kUnitRing;
+  if (!wait_parity_cluster(&bars->unit_empty[slot], (use & 1u) ^ 1u, abort, timeout_ns)) return false;
+  for (uint32_t dst = 0; dst < 2; ++dst) {
+    st_cluster_u32(mapa_shared(smem_u32(&bars->unit_id[slot]), dst), uint32_t(vc));
+    mbar_arrive_release_cluster(mapa_shared(smem_u32(&bars->unit_full[slot]), dst));
+  }
+  return true;
+}
+// Next unit for a reader: the unit index, -1 when none is left, -2 on abort or timeout.
+__device__ __forceinline__ int ring_take(Bars* bars, uint32_t lead_unit_empty0, uint32_t k, volatile int* abort,
+                                         uint64_t timeout_ns) {
+  const int slot = int(k % kUnitRing);
+  if (!wait_parity_cluster(&bars->unit_full[slot], (k / kUnitRing) & 1u, abort, timeout_ns)) return -2;
+  const int vc = *reinterpret_cast<volatile int*>(&bars->unit_id[slot]);
+  mbar_arrive_release_cluster(lead_unit_empty0 + uint32_t(slot) * 8u);
+  return vc;
+}
+
+static_assert(sizeof(Bars) <= 512, "barrier block of 512 bytes");
 
 struct SubTile {
   int head;
@@ -587,6 +634,65 @@ static_assert(PairCfg::kSmem <= 232448, "227 KB of shared memory per CTA");
 constexpr uint32_t kPairRegsSoftmax = 192, kPairRegsOther = 120;
 static_assert(2 * kPairRegsSoftmax + kPairRegsOther <= 3 * 168, "register split exceeds the launch's registers");
 
+// One work unit of the pair kernel (one cluster of the grid): unit index vc ->
+// work item, this CTA's two sub-tiles and the K/V range they share.  Units are
+// numbered in chunks of work items (longest first), K/V-head-major inside a
+// chunk, so that clusters running at the same time stream the same K/V tiles
+// through L2.
+// Heads mode (GQA group a multiple of 4): a unit is a quad of query heads of
+// one K/V head and one row tile; CTA rank r takes heads 4u + 2r, 4u + 2r + 1.
+// Rows mode (any other group): a unit is one query head and a quad of row
+// tiles; CTA rank r takes row tiles 4t + 2r and 4t + 2r + 1.
+struct PairUnit {
+  HalfDesc hd;
+  SubTile st[2];
+  int n;              // K/V tiles every sub-tile of the unit visits (they share each MMA)
+  int kv_end, kv_head;
+  int64_t row_base;   // Q/O row of the half's row 0
+};
+
+__device__ __forceinline__ PairUnit pair_unit(const Params& p, int vc, uint32_t rank) {
+  const int units_per_kv = p.pair_rows ? p.group : (p.groups_per_kv >> 1);
+  const int per_chunk = p.chunk_items * (p.pair_rows ? p.h_q : (p.head_groups >> 1));
+  const int chunk = vc / per_chunk;
+  const int r = vc - chunk * per_chunk;
+  const int w_items = min(p.chunk_items, p.n_items - chunk * p.chunk_items);
+  const int kvh = r / (w_items * units_per_kv);
+  const int r2 = r - kvh * w_items * units_per_kv;
+  const int item_idx = chunk * p.chunk_items + r2 / units_per_kv;
+  const int unit = kvh * units_per_kv + r2 % units_per_kv;
+  const WorkItem w = p.items[item_idx];
+  PairUnit u;
+  u.hd = p.halves[w.half_id];
+  if (p.pair_rows) {
+    u.st[0] = {unit, (4 * w.tile + 2 * int(rank)) * 128, 0};
+    u.st[1] = {unit, (4 * w.tile + 2 * int(rank) + 1) * 128, 0};
+    // the keys of the quad's last valid row tile; lower rows see the extra
+    // tiles fully masked (P = 0), rows past the half are computed and not written
+    const int last_tile = min(4 * w.tile + 3, (u.hd.lq - 1) / 128);
+    u.n = tiles_for(u.hd, last_tile * 128, p.causal);
+  } else {
+    u.st[0] = {4 * unit + 2 * int(rank), w.tile * 128, 0};
+    u.st[1] = {4 * unit + 2 * int(rank) + 1, w.tile * 128, 0};
+    u.n = tiles_for(u.hd, u.st[0].q0, p.causal);          // same rows, same keys
+  }
+  u.st[0].n = u.n;
+  u.st[1].n = u.n;
+  u.kv_end = p.causal ? u.hd.kv_len : u.hd.kv_full;
+  u.kv_head = u.st[0].head / p.group;
+  u.row_base = int64_t(u.hd.rank - p.rank_begin) * p.M + u.hd.row0;
+  return u;
+}
+
+// Persistent over units: a cluster does the unit of its own blockIdx, then
+// takes the units of clusters that have not started yet (cluster launch
+// control cancels their launch), until none is left.  The leader's producer
+// requests the next unit when it starts a unit and hands the answer to every
+// role through the unit ring.  All roles walk the same unit sequence, so the
+// barrier phases carry over from unit to unit (per-role counts of units, K/V
+// stages and tiles).  The next unit's Q is loaded as soon as the current
+// unit's last S MMAs have read Q (q_free), and its first S runs while the
+// current unit's last P.V and epilogue do.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -601,53 +707,14 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();     // 0: leader (issues the MMAs), 1: peer
   const bool leader = rank == 0;
-
-  // ---- work decomposition: clusters in chunks of items, K/V-head-major ----
-  // Heads mode (GQA group a multiple of 4): a unit is a quad of query heads of
-  // one K/V head and one row tile; CTA rank r takes heads 4u + 2r, 4u + 2r + 1.
-  // Rows mode (any other group): a unit is one query head and a quad of row
-  // tiles; CTA rank r takes row tiles 4t + 2r and 4t + 2r + 1.
-  int item_idx, unit;
-  {
-    const int cl = blockIdx.x >> 1;
-    const int units_per_kv = p.pair_rows ? p.group : (p.groups_per_kv >> 1);
-    const int per_chunk = p.chunk_items * (p.pair_rows ? p.h_q : (p.head_groups >> 1));
-    const int chunk = cl / per_chunk;
-    const int r = cl - chunk * per_chunk;
-    const int w_items = min(p.chunk_items, p.n_items - chunk * p.chunk_items);
-    const int kvh = r / (w_items * units_per_kv);
-    const int r2 = r - kvh * w_items * units_per_kv;
-    item_idx = chunk * p.chunk_items + r2 / units_per_kv;
-    unit = kvh * units_per_kv + r2 % units_per_kv;
-  }
-  const WorkItem w = p.items[item_idx];
-  const HalfDesc hd = p.halves[w.half_id];
-  SubTile st[2];
-  int n_all;   // K/V tiles every sub-tile of the cluster visits (they share each MMA)
-  if (p.pair_rows) {
-    st[0] = {unit, (4 * w.tile + 2 * int(rank)) * 128, 0};
-    st[1] = {unit, (4 * w.tile + 2 * int(rank) + 1) * 128, 0};
-    // the keys of the quad's last valid row tile; lower rows see the extra
-    // tiles fully masked (P = 0), rows past the half are computed and not written
-    const int last_tile = min(4 * w.tile + 3, (hd.lq - 1) / 128);
-    n_all = tiles_for(hd, last_tile * 128, p.causal);
-  } else {
-    st[0] = {4 * unit + 2 * int(rank), w.tile * 128, 0};
-    st[1] = {4 * unit + 2 * int(rank) + 1, w.tile * 128, 0};
-    n_all = tiles_for(hd, st[0].q0, p.causal);            // same rows, same keys
-  }
-  st[0].n = n_all;
-  st[1].n = n_all;
-  const int kv_end = p.causal ? hd.kv_len : hd.kv_full;
-  const int n_max = n_all;
-  const int kv_head = st[0].head / p.group;
-  const int64_t row_base = int64_t(hd.rank - p.rank_begin) * p.M + hd.row0;
+  const int vc0 = int(blockIdx.x >> 1);        // the cluster's first unit
 
   // ---- setup: barriers in both CTAs, TMEM for the pair, then a cluster barrier
   // so that no CTA signals the other's barriers before they exist ----
   if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full[0], 2);        // one expect_tx arrival from each CTA's producer (both Q tiles)
+    mbar_init(&bars->q_full[1], 1);        // q_free: the unit's last S MMAs have read Q (commit)
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->q_full[i], 2);      // one expect_tx arrival from each CTA's producer
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->p_full[i], 256);    // 128 softmax threads of each CTA
       mbar_init(&bars->o_full[i], 1);
@@ -657,6 +724,12 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_init(&bars->kv_full[s], 2);     // one expect_tx arrival from each CTA's producer
       mbar_init(&bars->kv_empty[s], 1);
     }
+    for (int i = 0; i < kUnitRing; ++i) {
+      mbar_init(&bars->unit_full[i], 1);
+      mbar_init(&bars->unit_empty[i], kUnitReaders);
+    }
+    mbar_init(&bars->clc_full, 1);
+    bars->clc_issued = 0;
     bars->abort = (p.status && (*reinterpret_cast<volatile int*>(p.status) & kStatusTimeout)) ? 1 : 0;
     fence_barrier_init();
   }
@@ -674,123 +747,160 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  uint64_t* q_full = &bars->q_full[0];
+  uint64_t* q_free = &bars->q_full[1];
   // The leader's barriers, as shared::cluster addresses (the peer signals them remotely).
-  const uint32_t lead_q_full0 = mapa_shared(smem_u32(&bars->q_full[0]), 0);
+  const uint32_t lead_q_full = mapa_shared(smem_u32(q_full), 0);
   const uint32_t lead_kv_full0 = mapa_shared(smem_u32(&bars->kv_full[0]), 0);
   const uint32_t lead_p_full0 = mapa_shared(smem_u32(&bars->p_full[0]), 0);
+  const uint32_t lead_unit_empty0 = mapa_shared(smem_u32(&bars->unit_empty[0]), 0);
+  uint32_t clc_read = 0;   // cancel responses read (the leader's producer)
 
   if (warp >= 8) {
   regs_dec<kPairRegsOther>();
   if (warp == kWarpLoad) {
     // ================= TMA producer (both CTAs: this CTA's halves) =================
-    const int32_t* pt = p.page_table + int64_t(hd.seq) * p.max_pages;
-    bool q_issued[2] = {false, false};
-    if (lane == 0 && !*abort) {
-      for (int i = 0; i < 2; ++i) {
-        if (n_max == 0) continue;
-        q_issued[i] = true;
-        uint8_t* dst = smem + C::kQOff + i * C::kQBytes;
-        const uint32_t bar = lead_q_full0 + uint32_t(i) * 8u;
-        mbar_arrive_expect_tx_cluster(bar, C::kQBytes);
-        for (int b = 0; b < 2; ++b)
-          tma_load_3d_pair(dst + b * C::kBoxBytes, &tm_q, bar, b * 64, st[i].head, int32_t(row_base + st[i].q0));
-      }
-    }
     const int kbox = p.box_rows < 64 ? p.box_rows : 64;       // K half: 64 keys
     const int vbox = p.box_rows;                              // V half: 128 keys
     const int kchunks = 64 / kbox, vchunks = 128 / vbox;
     bool bad_page = false;
-    // Stage t (t = 0 .. n_max): this CTA's half of K_t if t < n_max, of V_{t-1} if t >= 1.
-    int t = 0;
-    for (; t <= n_max && !*abort; ++t) {
-      const int slot = t % C::kStages;
-      const uint32_t use = t / C::kStages;
-      if (!wait_parity(&bars->kv_empty[slot], (use & 1u) ^ 1u, abort, p.timeout_ns)) break;
-      uint8_t* stage = smem + C::kKVOff + slot * C::kStageBytes;
-      uint8_t* ktile = stage;
-      uint8_t* vtile = stage + C::kKHalfBytes;
-      const bool has_k = t < n_max, has_v = t >= 1;
-      const int key0k = t * 128 + 64 * int(rank);           // first key of this CTA's K half
-      const int key0v = (t - 1) * 128;                       // first key of the V tile
-      uint32_t tma_bytes = 0;
-      bool manual = false;
-      if (has_k)
-        for (int c = 0; c < kchunks; ++c) {
-          if (key0k + (c + 1) * kbox <= kv_end) tma_bytes += kbox * 128 * 2;
-          else manual = true;
+    int tg = 0;               // K/V stages issued so far (all units)
+    uint32_t qk = 0;          // units whose Q was issued
+    uint32_t ring_k = 0;      // unit-ring entries written (leader) or taken (peer)
+    uint32_t clc_ph = 0;      // phase of clc_full
+    uint32_t clc_taken = 0;   // cancel responses read
+    int vc = vc0;
+    while (vc >= 0) {
+      if (__any_sync(0xffffffffu, *abort != 0)) break;
+      const PairUnit u = pair_unit(p, vc, rank);
+      bool ok = true;
+      if (u.n > 0) {
+        const int32_t* pt = p.page_table + int64_t(u.hd.seq) * p.max_pages;
+        // Q of both sub-tiles (the previous unit's last S MMAs have read the old Q).
+        if (lane == 0) {
+          mbar_arrive_expect_tx_cluster(lead_q_full, 2 * C::kQBytes);
+          for (int i = 0; i < 2; ++i)
+            for (int b = 0; b < 2; ++b)
+              tma_load_3d_pair(smem + C::kQOff + i * C::kQBytes + b * C::kBoxBytes, &tm_q, lead_q_full, b * 64,
+                               u.st[i].head, int32_t(u.row_base + u.st[i].q0));
         }
-      if (has_v)
-        for (int c = 0; c < vchunks; ++c) {
-          if (key0v + (c + 1) * vbox <= kv_end) tma_bytes += vbox * 128;
-          else manual = true;
-        }
-      if (manual) {
-        // Rows at or beyond kv_len are filled by hand (real keys copied, the rest zero).
-        for (int which = 0; which < 2; ++which) {
-          if (which == 0 && !has_k) continue;
-          if (which == 1 && !has_v) continue;
-          const int rows = which == 0 ? 64 : 128, box = which == 0 ? kbox : vbox;
-          const int units_per_row = which == 0 ? 16 : 8;     // 16-byte pieces of this CTA's part of a row
-          const int key0 = which == 0 ? key0k : key0v;
-          const __nv_bfloat16* pool = which == 0 ? p.k_pool : p.v_pool;
-          for (int c = 0; c < rows / box; ++c) {
-            if (key0 + (c + 1) * box <= kv_end) continue;
-            for (int u = lane; u < box * units_per_row; u += 32) {
-              const int row = c * box + u / units_per_row;
-              const int rem = u % units_per_row;
-              const int b = rem >> 3, ch = rem & 7;          // column box (K only) and 16-byte piece
-              const int key = key0 + row;
-              const int col = which == 0 ? b * 64 + ch * 8 : 64 * int(rank) + ch * 8;
-              int4 v = make_int4(0, 0, 0, 0);
-              if (key < kv_end) {
-                const int64_t slot_id = int64_t(__ldg(pt + key / p.page_size)) * p.page_size + key % p.page_size;
-                if (slot_id >= 0 && slot_id < p.num_slots)
-                  v = __ldg(reinterpret_cast<const int4*>(pool + (slot_id * p.h_kv + kv_head) * D + col));
-                else
-                  bad_page = true;
+        __syncwarp();
+        ++qk;
+        // Stage t of the unit (t = 0 .. n): this CTA's half of K_t if t < n, of V_{t-1} if t >= 1.
+        for (int t = 0; t <= u.n; ++t, ++tg) {
+          const int slot = tg % C::kStages;
+          const uint32_t use = tg / C::kStages;
+          ok = __all_sync(0xffffffffu, wait_parity(&bars->kv_empty[slot], (use & 1u) ^ 1u, abort, p.timeout_ns));
+          if (!ok) break;
+          uint8_t* stage = smem + C::kKVOff + slot * C::kStageBytes;
+          uint8_t* ktile = stage;
+          uint8_t* vtile = stage + C::kKHalfBytes;
+          const bool has_k = t < u.n, has_v = t >= 1;
+          const int key0k = t * 128 + 64 * int(rank);           // first key of this CTA's K half
+          const int key0v = (t - 1) * 128;                       // first key of the V tile
+          uint32_t tma_bytes = 0;
+          bool manual = false;
+          if (has_k)
+            for (int c = 0; c < kchunks; ++c) {
+              if (key0k + (c + 1) * kbox <= u.kv_end) tma_bytes += kbox * 128 * 2;
+              else manual = true;
+            }
+          if (has_v)
+            for (int c = 0; c < vchunks; ++c) {
+              if (key0v + (c + 1) * vbox <= u.kv_end) tma_bytes += vbox * 128;
+              else manual = true;
+            }
+          if (manual) {
+            // Rows at or beyond kv_len are filled by hand (real keys copied, the rest zero).
+            for (int which = 0; which < 2; ++which) {
+              if (which == 0 && !has_k) continue;
+              if (which == 1 && !has_v) continue;
+              const int rows = which == 0 ? 64 : 128, box = which == 0 ? kbox : vbox;
+              const int units_per_row = which == 0 ? 16 : 8;   // 16-byte pieces of this CTA's part of a row
+              const int key0 = which == 0 ? key0k : key0v;
+              const __nv_bfloat16* pool = which == 0 ? p.k_pool : p.v_pool;
+              for (int c = 0; c < rows / box; ++c) {
+                if (key0 + (c + 1) * box <= u.kv_end) continue;
+                for (int e = lane; e < box * units_per_row; e += 32) {
+                  const int row = c * box + e / units_per_row;
+                  const int rem = e % units_per_row;
+                  const int b = rem >> 3, ch = rem & 7;        // column box (K only) and 16-byte piece
+                  const int key = key0 + row;
+                  const int col = which == 0 ? b * 64 + ch * 8 : 64 * int(rank) + ch * 8;
+                  int4 v = make_int4(0, 0, 0, 0);
+                  if (key < u.kv_end) {
+                    const int64_t slot_id =
+                        int64_t(__ldg(pt + key / p.page_size)) * p.page_size + key % p.page_size;
+                    if (slot_id >= 0 && slot_id < p.num_slots)
+                      v = __ldg(reinterpret_cast<const int4*>(pool + (slot_id * p.h_kv + u.kv_head) * D + col));
+                    else
+                      bad_page = true;
+                  }
+                  uint8_t* dstp = which == 0 ? ktile + b * (64 * 128) : vtile;
+                  *reinterpret_cast<int4*>(dstp + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+                }
               }
-              uint8_t* dstp = which == 0 ? ktile + b * (64 * 128) : vtile;
-              *reinterpret_cast<int4*>(dstp + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+          const uint32_t bar = lead_kv_full0 + uint32_t(slot) * 8u;
+          if (lane == 0) mbar_arrive_expect_tx_cluster(bar, tma_bytes);
+          __syncwarp();
+          // One lane per page chunk: K chunks first, then V chunks.
+          const int nk = has_k ? kchunks : 0, nv = has_v ? vchunks : 0;
+          for (int e = lane; e < nk + nv; e += 32) {
+            const bool is_k = e < nk;
+            const int c = is_k ? e : e - nk;
+            const int box = is_k ? kbox : vbox;
+            const int kc = (is_k ? key0k : key0v) + c * box;
+            if (kc + box > u.kv_end) continue;
+            const int32_t page = __ldg(pt + kc / p.page_size);
+            const bool in_pool = uint32_t(page) < uint32_t(p.num_pages);
+            bad_page |= !in_pool;
+            const int32_t slot0 = (in_pool ? page : p.num_pages) * p.page_size + kc % p.page_size;
+            if (is_k) {
+              for (int b = 0; b < 2; ++b)
+                tma_load_3d_pair(ktile + b * (64 * 128) + c * box * 128, &tm_k, bar, b * 64, u.kv_head, slot0);
+            } else {
+              tma_load_3d_pair(vtile + c * box * 128, &tm_v, bar, 64 * int(rank), u.kv_head, slot0);
             }
           }
+          __syncwarp();
         }
-        fence_proxy_async_smem();
-        __syncwarp();
+        if (!ok) break;
+        // The unit's last S MMAs have read Q: the next unit's Q may be loaded.
+        ok = __all_sync(0xffffffffu, wait_parity(q_free, (qk - 1) & 1u, abort, p.timeout_ns));
+        if (!ok) break;
       }
-      const uint32_t bar = lead_kv_full0 + uint32_t(slot) * 8u;
-      if (lane == 0) mbar_arrive_expect_tx_cluster(bar, tma_bytes);
-      __syncwarp();
-      // One lane per page chunk: K chunks first, then V chunks.
-      const int nk = has_k ? kchunks : 0, nv = has_v ? vchunks : 0;
-      for (int u = lane; u < nk + nv; u += 32) {
-        const bool is_k = u < nk;
-        const int c = is_k ? u : u - nk;
-        const int box = is_k ? kbox : vbox;
-        const int kc = (is_k ? key0k : key0v) + c * box;
-        if (kc + box > kv_end) continue;
-        const int32_t page = __ldg(pt + kc / p.page_size);
-        const bool in_pool = uint32_t(page) < uint32_t(p.num_pages);
-        bad_page |= !in_pool;
-        const int32_t slot0 = (in_pool ? page : p.num_pages) * p.page_size + kc % p.page_size;
-        if (is_k) {
-          for (int b = 0; b < 2; ++b)
-            tma_load_3d_pair(ktile + b * (64 * 128) + c * box * 128, &tm_k, bar, b * 64, kv_head, slot0);
+      // The next unit: the leader reads the answer to the MMA thread's cancel
+      // request and hands it on, the peer takes it from the ring.
+      int nxt = -2;
+      if (lane == 0) {
+        if (leader) {
+          if (wait_parity(&bars->clc_full, clc_ph, abort, p.timeout_ns)) {
+            clc_ph ^= 1u;
+            ++clc_taken;
+            const int x = clc_first_ctaid_x(bars->clc_resp);
+            fence_proxy_async_smem();          // the next response is written through the async proxy
+            nxt = x < 0 ? -1 : (x >> 1);
+            if (!ring_put(bars, ring_k++, nxt, abort, p.timeout_ns)) nxt = -2;
+          }
         } else {
-          tma_load_3d_pair(vtile + c * box * 128, &tm_v, bar, 64 * int(rank), kv_head, slot0);
+          nxt = ring_take(bars, lead_unit_empty0, ring_k++, abort, p.timeout_ns);
         }
       }
-      __syncwarp();
+      vc = __shfl_sync(0xffffffffu, nxt, 0);
     }
-    const int load_no = t;
     if (bad_page && p.status) atomicOr(p.status, kStatusBadPage);
     // Copies of both CTAs land on the leader's barriers: the leader's producer
     // drains them; the cluster barrier at the end keeps the peer alive until then.
     if (lane == 0 && leader) {
-      for (int n = max(0, load_no - C::kStages); n < load_no; ++n)
-        drain_parity(&bars->kv_full[n % C::kStages], (uint32_t(n / C::kStages)) & 1u, p.timeout_ns);
-      for (int i = 0; i < 2; ++i)
-        if (q_issued[i]) drain_parity(&bars->q_full[i], 0, p.timeout_ns);
+      for (int k = max(0, tg - C::kStages); k < tg; ++k)
+        drain_parity(&bars->kv_full[k % C::kStages], (uint32_t(k / C::kStages)) & 1u, p.timeout_ns);
+      if (qk > 0) drain_parity(q_full, (qk - 1) & 1u, p.timeout_ns);
     }
+    clc_read = clc_taken;
   } else if (warp == kWarpMma && leader) {
     // ================= MMA issue (leader CTA, one thread) =================
     if (lane == 0) {
@@ -818,33 +928,60 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           mma_ts_pair(tmem + col_o, tmem + col_p + kk * 8, dv + uint64_t((kk * 2048) >> 4), idesc_o,
                       (acc || kk > 0) ? 1u : 0u);
       };
-      const int n = n_max;
-      bool ok = n > 0;
-      if (ok) ok = wait_parity(&bars->q_full[0], 0, abort, p.timeout_ns);
-      if (ok) ok = wait_parity(&bars->q_full[1], 0, abort, p.timeout_ns);
-      if (ok) ok = wait_parity(&bars->kv_full[0], 0, abort, p.timeout_ns);   // stage 0: K_0
-      if (ok) {
-        tc_fence_after();
-        issue_s(C::kColS0, dq0, 0); mma_commit_pair(&bars->s_full[0], both);
-        issue_s(C::kColS1, dq1, 0); mma_commit_pair(&bars->s_full[1], both);
-        mma_commit_pair(&bars->kv_empty[0], both);
+      int tg = 0;            // K/V stages consumed so far (all units)
+      uint32_t qk = 0;       // units started
+      uint32_t jg = 0;       // tiles of all earlier units (phase base of p_full)
+      uint32_t ring_k = 0;   // unit-ring entries taken
+      uint32_t issued = 0;   // cancel requests issued
+      auto request_next = [&]() {
+        mbar_arrive_expect_tx(&bars->clc_full, 16);
+        clc_try_cancel(bars->clc_resp, &bars->clc_full);
+        ++issued;
+      };
+      bool ok = true;
+      for (int vc = vc0; vc >= 0 && ok;) {
+        const int n = pair_unit(p, vc, 0).n;
+        const int req_j = n - 2 - kClcLead;   // loop iteration after which to ask (-1: after the first S)
+        if (n <= 0) request_next();
+        if (n > 0) {
+          if (!(ok = wait_parity(q_full, qk & 1u, abort, p.timeout_ns))) break;
+          {
+            const int slot = tg % C::kStages;                 // stage 0 of the unit: K_0
+            if (!(ok = wait_parity(&bars->kv_full[slot], uint32_t(tg / C::kStages) & 1u, abort, p.timeout_ns)))
+              break;
+            tc_fence_after();
+            issue_s(C::kColS0, dq0, slot); mma_commit_pair(&bars->s_full[0], both);
+            issue_s(C::kColS1, dq1, slot); mma_commit_pair(&bars->s_full[1], both);
+            if (n == 1) mma_commit_pair(q_free, both);        // the unit's last S
+            mma_commit_pair(&bars->kv_empty[slot], both);
+            ++tg;
+            if (req_j < 0) request_next();
+          }
+          for (int j = 0; j < n && ok; ++j, ++tg) {
+            const int slot = tg % C::kStages;                 // stage with V_j and K_{j+1}
+            const uint32_t ph = (jg + uint32_t(j)) & 1u;
+            if (!(ok = wait_parity(&bars->kv_full[slot], uint32_t(tg / C::kStages) & 1u, abort, p.timeout_ns)))
+              break;
+            if (!(ok = wait_spin(&bars->p_full[0], ph, abort, p.timeout_ns))) break;
+            tc_fence_after();
+            issue_pv(C::kColO0, C::kColS0, slot, j > 0);
+            if (j == n - 1) mma_commit_pair(&bars->o_full[0], both);
+            else { issue_s(C::kColS0, dq0, slot); mma_commit_pair(&bars->s_full[0], both); }
+            if (!(ok = wait_spin(&bars->p_full[1], ph, abort, p.timeout_ns))) break;
+            tc_fence_after();
+            issue_pv(C::kColO1, C::kColS1, slot, j > 0);
+            if (j == n - 1) mma_commit_pair(&bars->o_full[1], both);
+            else { issue_s(C::kColS1, dq1, slot); mma_commit_pair(&bars->s_full[1], both); }
+            if (j == n - 2) mma_commit_pair(q_free, both);    // the unit's last S
+            mma_commit_pair(&bars->kv_empty[slot], both);
+            if (j == req_j) request_next();
+          }
+          jg += uint32_t(n);
+          ++qk;
+        }
+        if (ok) vc = ring_take(bars, lead_unit_empty0, ring_k++, abort, p.timeout_ns);
       }
-      for (int j = 0; j < n && ok; ++j) {
-        const int t = j + 1;                    // stage with V_j and K_{j+1}
-        const int slot = t % C::kStages;
-        if (!(ok = wait_parity(&bars->kv_full[slot], uint32_t(t / C::kStages) & 1u, abort, p.timeout_ns))) break;
-        if (!(ok = wait_spin(&bars->p_full[0], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
-        tc_fence_after();
-        issue_pv(C::kColO0, C::kColS0, slot, j > 0);
-        if (j == n - 1) mma_commit_pair(&bars->o_full[0], both);
-        else { issue_s(C::kColS0, dq0, slot); mma_commit_pair(&bars->s_full[0], both); }
-        if (!(ok = wait_spin(&bars->p_full[1], uint32_t(j) & 1u, abort, p.timeout_ns))) break;
-        tc_fence_after();
-        issue_pv(C::kColO1, C::kColS1, slot, j > 0);
-        if (j == n - 1) mma_commit_pair(&bars->o_full[1], both);
-        else { issue_s(C::kColS1, dq1, slot); mma_commit_pair(&bars->s_full[1], both); }
-        mma_commit_pair(&bars->kv_empty[slot], both);
-      }
+      bars->clc_issued = issued;
       mma_commit_pair(&bars->mma_done, 1);
       drain_parity(&bars->mma_done, 0, p.timeout_ns);
     }
@@ -854,69 +991,90 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // ================= softmax + epilogue (warps 0-7, both CTAs) =================
     regs_inc<kPairRegsSoftmax>();
     const int g = warp >> 2;
-    const SubTile& me = st[g];
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t t_s = tmem + lane_off + (g ? C::kColS1 : C::kColS0);
     const uint32_t t_o = tmem + lane_off + (g ? C::kColO1 : C::kColO0);
     const uint32_t p_full_lead = lead_p_full0 + uint32_t(g) * 8u;
-    const int q_row = me.q0 + r;
-    const int my_pos = p.causal ? hd.kv_pos0 + q_row : hd.kv_full - 1;
-    const int first_pos = p.causal ? hd.kv_pos0 + me.q0 : hd.kv_full - 1;
-    float m = -CUDART_INF_F, l = 0.f;
-    bool ok = me.n > 0;
-    for (int j = 0; j < me.n && ok; ++j) {
-      ok = wait_parity(&bars->s_full[g], uint32_t(j) & 1u, abort, p.timeout_ns);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // TMEM access below is warp-wide
-      tc_fence_after();
-      uint32_t sr[128];
+    uint32_t qk = 0;       // units done
+    uint32_t jg = 0;       // tiles of all earlier units
+    uint32_t ring_k = 0;   // unit-ring entries taken
+    int vc = vc0;
+    while (vc >= 0) {
+      const PairUnit u = pair_unit(p, vc, rank);
+      const int my_head = g ? u.st[1].head : u.st[0].head;   // no dynamic index: u stays in registers
+      const int my_q0 = g ? u.st[1].q0 : u.st[0].q0;
+      const int n = u.n;
+      if (n > 0) {
+        const int q_row = my_q0 + r;
+        const int my_pos = p.causal ? u.hd.kv_pos0 + q_row : u.hd.kv_full - 1;
+        const int first_pos = p.causal ? u.hd.kv_pos0 + my_q0 : u.hd.kv_full - 1;
+        float m = -CUDART_INF_F, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n && ok; ++j) {
+          ok = wait_parity(&bars->s_full[g], (jg + uint32_t(j)) & 1u, abort, p.timeout_ns);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // TMEM access below is warp-wide
+          tc_fence_after();
+          uint32_t sr[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-      tmem_wait_ld();
-      const bool masked = j * 128 + 127 > first_pos;
-      if (masked) {
-        const int limit = my_pos - j * 128 + 1;
+          for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+          tmem_wait_ld();
+          const bool masked = j * 128 + 127 > first_pos;
+          if (masked) {
+            const int limit = my_pos - j * 128 + 1;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= limit) sr[c] = 0xFF800000u;
-      }
-      softmax_tile<D>(sr, j, masked, p.scale_log2, t_s, t_o, m, l);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive_cluster(p_full_lead);         // the leader's barrier, from either CTA
-    }
-    if (ok) ok = wait_parity(&bars->o_full[g], 0, abort, p.timeout_ns);
-    ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-wide
-    if (ok) {
-      tc_fence_after();
-      const bool valid = q_row < hd.lq;
-      const int64_t grow = row_base + q_row;
-      const float inv = 1.f / l;
-      __nv_bfloat16* op = p.out + (grow * p.h_q + me.head) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(t_o + c * 32, o);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        if (valid) {
-          int4* dst = reinterpret_cast<int4*>(op + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_int4(int(pk[4 * v]), int(pk[4 * v + 1]), int(pk[4 * v + 2]), int(pk[4 * v + 3]));
+            for (int c = 0; c < 128; ++c)
+              if (c >= limit) sr[c] = 0xFF800000u;
+          }
+          softmax_tile<D>(sr, j, masked, p.scale_log2, t_s, t_o, m, l);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive_cluster(p_full_lead);       // the leader's barrier, from either CTA
         }
+        if (ok) ok = wait_parity(&bars->o_full[g], qk & 1u, abort, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) break;  // the TMEM loads below are warp-wide
+        // Epilogue.  Its TMEM loads complete (wait::ld) before this warp writes
+        // the next unit's P, so the next unit's first P.V (which overwrites O)
+        // cannot race them.
+        tc_fence_after();
+        const bool valid = q_row < u.hd.lq;
+        const int64_t grow = u.row_base + q_row;
+        const float inv = 1.f / l;
+        __nv_bfloat16* op = p.out + (grow * p.h_q + my_head) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          if (valid) {
+            int4* dst = reinterpret_cast<int4*>(op + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_int4(int(pk[4 * v]), int(pk[4 * v + 1]), int(pk[4 * v + 2]), int(pk[4 * v + 3]));
+          }
+        }
+        if (valid && p.lse) p.lse[grow * p.h_q + my_head] = (m + log2f(l)) * 0.69314718055994531f;
+        jg += uint32_t(n);
+        ++qk;
       }
-      if (valid && p.lse) p.lse[grow * p.h_q + me.head] = (m + log2f(l)) * 0.69314718055994531f;
+      int nxt = -2;
+      if (lane == 0) nxt = ring_take(bars, lead_unit_empty0, ring_k++, abort, p.timeout_ns);
+      vc = __shfl_sync(0xffffffffu, nxt, 0);
     }
   }
 
   // ---- teardown: both CTAs done with TMEM and with each other's barriers ----
   tc_fence_before();
   __syncthreads();
+  // A cancel response still in flight (only after an abort: one request at
+  // most is outstanding) lands before this CTA's shared memory is released.
+  if (leader && warp == kWarpLoad && lane == 0 && bars->clc_issued > clc_read)
+    drain_parity(&bars->clc_full, clc_read & 1u, p.timeout_ns);
   cluster_sync();
   if (warp == kWarpMma) {
     tc_fence_after();

@@ -191,6 +191,64 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar_clust
                : "memory");
 }
 
+// Cluster launch control (sm_100): try_cancel asks the hardware scheduler to
+// cancel the launch of one cluster of this grid that has not started yet; the
+// 16-byte response (written to this CTA's shared memory, completion counted
+// on an mbarrier) says whether it succeeded and, if so, the first CTA index of
+// that cluster, whose work this cluster then does.  After a failed request no
+// further one may be issued.
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+  asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+               ::"r"(smem_u32(resp)), "r"(smem_u32(bar)) : "memory");
+}
+// x index of the first CTA of the cancelled cluster, or -1 if the request failed.
+__device__ __forceinline__ int clc_first_ctaid_x(const void* resp) {
+  int x;
+  asm volatile(
+      "{\n\t.reg .b128 r;\n\t.reg .pred ok;\n\t"
+      "ld.shared.b128 r, [%1];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 ok, r;\n\t"
+      "mov.s32 %0, -1;\n\t"
+      "@ok clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %0, r;\n\t}"
+      : "=r"(x)
+      : "r"(smem_u32(resp))
+      : "memory");
+  return x;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Arrive with cluster-scope release: this thread's earlier shared-memory
+// accesses (the peer CTA's too) are visible to whoever observes the phase.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_acquire_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// wait_parity with cluster-scope acquire (the phase was completed from the other CTA).
+__device__ __forceinline__ bool wait_parity_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                    uint64_t timeout_ns) {
+  if (mbar_try_wait_acquire_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_acquire_cluster(bar, parity)) return true;
+    if (*abort) return false;
+    if ((it & 255u) == 0 && global_timer_ns() - t0 > timeout_ns) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // 3-D tiled TMA load into this CTA's shared memory whose completion bytes are
 // counted on a barrier of either CTA of the pair (shared::cluster address).
 __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const void* tmap, uint32_t bar_cluster,

@@ -953,7 +953,7 @@ def rerange_standalone(torch, zz, synth, dev, reps: int = 24, sets: int = 4, wit
     res["bytes_per_launch"] = nbytes
     res["method"] = (f"{reps} launches over {sets} rotating 268 MB buffer sets (cold L2), captured in one "
                      "CUDA graph; median of 5 replays")
-    res["roofline"] = {"bound": "hbm", "kernel": "move_rows_kernel (rerange)", "achieved": best,
+    res["roofline"] = {"bound": "hbm", "kernel": "move_rows_bulk (rerange, 2 KB rows)", "achieved": best,
                        "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                        "frac": best / float(peaks["hbm_gbs"]), "peak_source": f"{src} hbm_gbs",
                        "traffic": load_traffic("rerange_standalone")}

@@ -112,6 +112,39 @@ def test_single_rank_launches_match_full_launch():
         assert torch.equal(out_r[:n], full[r * p.M: r * p.M + n])
 
 
+def test_concurrent_launches_sharing_a_plan_are_bit_identical():
+    """Launches on two streams that share one plan and its workspace, running at
+    the same time, each give exactly the output of a launch run alone: the
+    persistent kernel hands out work units per launch (no shared counter), and
+    every unit is computed once in a fixed order.  Several waves of units, so
+    units are handed out while the other launch is running."""
+    run = Run(Case(4, [4096], 32, 4, 128, page_size=16))
+    p = run.ref_plan
+    q_sets = [run.q_ranked, (run.q_ranked * -0.75).contiguous()]
+    ref = []
+    for q in q_sets:
+        o = torch.full_like(q, float("nan"))
+        zz.attn_prefill(run.plan, q, run.k_pool, run.v_pool, run.page_table, 16, o,
+                        softmax_scale=run.softmax_scale)
+        torch.cuda.synchronize()
+        ref.append(o)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [[torch.full_like(q_sets[i], float("nan")) for _ in range(4)] for i in range(2)]
+    torch.cuda.synchronize()
+    for k in range(4):
+        for i in range(2):
+            zz.attn_prefill(run.plan, q_sets[i], run.k_pool, run.v_pool, run.page_table, 16, outs[i][k],
+                            softmax_scale=run.softmax_scale, stream=streams[i])
+    torch.cuda.synchronize()
+    valid = torch.cat([torch.arange(r * p.M, r * p.M + p.per_rank_actual_token[r]) for r in range(p.cp_size)])
+    valid = valid.to(run.out.device)
+    for i in range(2):
+        assert torch.isfinite(ref[i].index_select(0, valid).float()).all()
+        for k in range(4):
+            assert torch.equal(outs[i][k].index_select(0, valid), ref[i].index_select(0, valid)), (i, k)
+    assert run.plan.device_status() == 0
+
+
 def test_union_in_token_order_equals_unsharded_attention():
     """Outputs of all ranks, moved back to token order, equal plain causal attention."""
     from oracle import attention as OA

@@ -26,6 +26,7 @@ CASES = [
     (2, [32768], 8, 128, "bf16", 16),                     # the standalone rerange shape
     (4, [32768], 8, 128, "bf16", 16),
     (8, [32768], 8, 128, "bf16", 16),
+    (2, [3000, 77], 32, 128, "bf16", 16),                 # 8 KB rows, ragged ends of the CTA ranges
 ]
 
 
@@ -78,13 +79,14 @@ def test_shard_rows_bit_exact(cp, lens):
         assert (got[r * ref.M + n:(r + 1) * ref.M] == -1).all()   # padding untouched
 
 
-def test_rerange_k_only_and_out_of_range_slots_skipped():
+@pytest.mark.parametrize("h_kv,d", [(1, 64), (8, 128)], ids=["vector-copy", "bulk-copy"])
+def test_rerange_k_only_and_out_of_range_slots_skipped(h_kv, d):
     cp, lens = 2, [64]
     plan = zz.Plan(cp, extend_lens=lens)
     plan.upload()
     ref = OP.build_metadata(cp, 64, extend_lens=lens)
-    kg = torch.randn(cp * plan.M, 1, 64).to(torch.bfloat16).cuda()
-    kp = torch.zeros(64, 1, 64, dtype=torch.bfloat16, device="cuda")
+    kg = torch.randn(cp * plan.M, h_kv, d).to(torch.bfloat16).cuda()
+    kp = torch.zeros(64, h_kv, d, dtype=torch.bfloat16, device="cuda")
     loc = torch.arange(64, dtype=torch.int64)
     loc[5] = 1000                                    # out of range: must be skipped
     loc[6] = -3
@@ -95,6 +97,7 @@ def test_rerange_k_only_and_out_of_range_slots_skipped():
     keep = [t for t in range(64) if t not in (5, 6)]
     assert np.array_equal(got[keep], nat[keep])
     assert (got[5] == 0).all() and (got[6] == 0).all()
+    assert plan.device_status() == 0
 
 
 @pytest.mark.parametrize("cp,lens,width,dtype", [(4, [37, 50, 8], 16, torch.int32),

@@ -686,13 +686,17 @@ __device__ __forceinline__ PairUnit pair_unit(const Params& p, int vc, uint32_t 
 
 // Persistent over units: a cluster does the unit of its own blockIdx, then
 // takes the units of clusters that have not started yet (cluster launch
-// control cancels their launch), until none is left.  The leader's producer
-// requests the next unit when it starts a unit and hands the answer to every
-// role through the unit ring.  All roles walk the same unit sequence, so the
-// barrier phases carry over from unit to unit (per-role counts of units, K/V
-// stages and tiles).  The next unit's Q is loaded as soon as the current
-// unit's last S MMAs have read Q (q_free), and its first S runs while the
-// current unit's last P.V and epilogue do.
+// control cancels their launch), until none is left.  The MMA thread asks for
+// the next unit a few tiles before the end of the current one; the leader's
+// producer reads the answer and hands it to every role through the unit ring.
+// All roles walk the same unit sequence, so the barrier phases carry over from
+// unit to unit (per-role counts of units, K/V stages and tiles).  Once the
+// producer has issued the current unit's stages it already loads the next
+// unit's first K/V stages into the slots the MMA frees, and the next unit's Q
+// as soon as the current unit's last S MMAs have read Q (q_free); the next
+// unit's first S then runs while the current unit's last P.V and epilogue do.
+// Every planned unit has rows (the planner emits only row tiles that start
+// inside their half), so n >= 1 for every unit; the producer relies on it.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -769,110 +773,111 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint32_t ring_k = 0;      // unit-ring entries written (leader) or taken (peer)
     uint32_t clc_ph = 0;      // phase of clc_full
     uint32_t clc_taken = 0;   // cancel responses read
-    int vc = vc0;
-    while (vc >= 0) {
-      if (__any_sync(0xffffffffu, *abort != 0)) break;
-      const PairUnit u = pair_unit(p, vc, rank);
-      bool ok = true;
-      if (u.n > 0) {
-        const int32_t* pt = p.page_table + int64_t(u.hd.seq) * p.max_pages;
-        // Q of both sub-tiles (the previous unit's last S MMAs have read the old Q).
-        if (lane == 0) {
-          mbar_arrive_expect_tx_cluster(lead_q_full, 2 * C::kQBytes);
-          for (int i = 0; i < 2; ++i)
-            for (int b = 0; b < 2; ++b)
-              tma_load_3d_pair(smem + C::kQOff + i * C::kQBytes + b * C::kBoxBytes, &tm_q, lead_q_full, b * 64,
-                               u.st[i].head, int32_t(u.row_base + u.st[i].q0));
+    // Stage t of unit u (t = 0 .. n) into ring slot `slot`: this CTA's half of
+    // K_t if t < n, of V_{t-1} if t >= 1 (the slot is free: kv_empty passed).
+    auto issue_stage = [&](const PairUnit& u, const int32_t* pt, int t, int slot) {
+      uint8_t* stage = smem + C::kKVOff + slot * C::kStageBytes;
+      uint8_t* ktile = stage;
+      uint8_t* vtile = stage + C::kKHalfBytes;
+      const bool has_k = t < u.n, has_v = t >= 1;
+      const int key0k = t * 128 + 64 * int(rank);           // first key of this CTA's K half
+      const int key0v = (t - 1) * 128;                       // first key of the V tile
+      uint32_t tma_bytes = 0;
+      bool manual = false;
+      if (has_k)
+        for (int c = 0; c < kchunks; ++c) {
+          if (key0k + (c + 1) * kbox <= u.kv_end) tma_bytes += kbox * 128 * 2;
+          else manual = true;
         }
-        __syncwarp();
-        ++qk;
-        // Stage t of the unit (t = 0 .. n): this CTA's half of K_t if t < n, of V_{t-1} if t >= 1.
-        for (int t = 0; t <= u.n; ++t, ++tg) {
-          const int slot = tg % C::kStages;
-          const uint32_t use = tg / C::kStages;
-          ok = __all_sync(0xffffffffu, wait_parity(&bars->kv_empty[slot], (use & 1u) ^ 1u, abort, p.timeout_ns));
-          if (!ok) break;
-          uint8_t* stage = smem + C::kKVOff + slot * C::kStageBytes;
-          uint8_t* ktile = stage;
-          uint8_t* vtile = stage + C::kKHalfBytes;
-          const bool has_k = t < u.n, has_v = t >= 1;
-          const int key0k = t * 128 + 64 * int(rank);           // first key of this CTA's K half
-          const int key0v = (t - 1) * 128;                       // first key of the V tile
-          uint32_t tma_bytes = 0;
-          bool manual = false;
-          if (has_k)
-            for (int c = 0; c < kchunks; ++c) {
-              if (key0k + (c + 1) * kbox <= u.kv_end) tma_bytes += kbox * 128 * 2;
-              else manual = true;
-            }
-          if (has_v)
-            for (int c = 0; c < vchunks; ++c) {
-              if (key0v + (c + 1) * vbox <= u.kv_end) tma_bytes += vbox * 128;
-              else manual = true;
-            }
-          if (manual) {
-            // Rows at or beyond kv_len are filled by hand (real keys copied, the rest zero).
-            for (int which = 0; which < 2; ++which) {
-              if (which == 0 && !has_k) continue;
-              if (which == 1 && !has_v) continue;
-              const int rows = which == 0 ? 64 : 128, box = which == 0 ? kbox : vbox;
-              const int units_per_row = which == 0 ? 16 : 8;   // 16-byte pieces of this CTA's part of a row
-              const int key0 = which == 0 ? key0k : key0v;
-              const __nv_bfloat16* pool = which == 0 ? p.k_pool : p.v_pool;
-              for (int c = 0; c < rows / box; ++c) {
-                if (key0 + (c + 1) * box <= u.kv_end) continue;
-                for (int e = lane; e < box * units_per_row; e += 32) {
-                  const int row = c * box + e / units_per_row;
-                  const int rem = e % units_per_row;
-                  const int b = rem >> 3, ch = rem & 7;        // column box (K only) and 16-byte piece
-                  const int key = key0 + row;
-                  const int col = which == 0 ? b * 64 + ch * 8 : 64 * int(rank) + ch * 8;
-                  int4 v = make_int4(0, 0, 0, 0);
-                  if (key < u.kv_end) {
-                    const int64_t slot_id =
-                        int64_t(__ldg(pt + key / p.page_size)) * p.page_size + key % p.page_size;
-                    if (slot_id >= 0 && slot_id < p.num_slots)
-                      v = __ldg(reinterpret_cast<const int4*>(pool + (slot_id * p.h_kv + u.kv_head) * D + col));
-                    else
-                      bad_page = true;
-                  }
-                  uint8_t* dstp = which == 0 ? ktile + b * (64 * 128) : vtile;
-                  *reinterpret_cast<int4*>(dstp + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
-                }
+      if (has_v)
+        for (int c = 0; c < vchunks; ++c) {
+          if (key0v + (c + 1) * vbox <= u.kv_end) tma_bytes += vbox * 128;
+          else manual = true;
+        }
+      if (manual) {
+        // Rows at or beyond kv_len are filled by hand (real keys copied, the rest zero).
+        for (int which = 0; which < 2; ++which) {
+          if (which == 0 && !has_k) continue;
+          if (which == 1 && !has_v) continue;
+          const int rows = which == 0 ? 64 : 128, box = which == 0 ? kbox : vbox;
+          const int units_per_row = which == 0 ? 16 : 8;   // 16-byte pieces of this CTA's part of a row
+          const int key0 = which == 0 ? key0k : key0v;
+          const __nv_bfloat16* pool = which == 0 ? p.k_pool : p.v_pool;
+          for (int c = 0; c < rows / box; ++c) {
+            if (key0 + (c + 1) * box <= u.kv_end) continue;
+            for (int e = lane; e < box * units_per_row; e += 32) {
+              const int row = c * box + e / units_per_row;
+              const int rem = e % units_per_row;
+              const int b = rem >> 3, ch = rem & 7;        // column box (K only) and 16-byte piece
+              const int key = key0 + row;
+              const int col = which == 0 ? b * 64 + ch * 8 : 64 * int(rank) + ch * 8;
+              int4 v = make_int4(0, 0, 0, 0);
+              if (key < u.kv_end) {
+                const int64_t slot_id =
+                    int64_t(__ldg(pt + key / p.page_size)) * p.page_size + key % p.page_size;
+                if (slot_id >= 0 && slot_id < p.num_slots)
+                  v = __ldg(reinterpret_cast<const int4*>(pool + (slot_id * p.h_kv + u.kv_head) * D + col));
+                else
+                  bad_page = true;
               }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-          }
-          const uint32_t bar = lead_kv_full0 + uint32_t(slot) * 8u;
-          if (lane == 0) mbar_arrive_expect_tx_cluster(bar, tma_bytes);
-          __syncwarp();
-          // One lane per page chunk: K chunks first, then V chunks.
-          const int nk = has_k ? kchunks : 0, nv = has_v ? vchunks : 0;
-          for (int e = lane; e < nk + nv; e += 32) {
-            const bool is_k = e < nk;
-            const int c = is_k ? e : e - nk;
-            const int box = is_k ? kbox : vbox;
-            const int kc = (is_k ? key0k : key0v) + c * box;
-            if (kc + box > u.kv_end) continue;
-            const int32_t page = __ldg(pt + kc / p.page_size);
-            const bool in_pool = uint32_t(page) < uint32_t(p.num_pages);
-            bad_page |= !in_pool;
-            const int32_t slot0 = (in_pool ? page : p.num_pages) * p.page_size + kc % p.page_size;
-            if (is_k) {
-              for (int b = 0; b < 2; ++b)
-                tma_load_3d_pair(ktile + b * (64 * 128) + c * box * 128, &tm_k, bar, b * 64, u.kv_head, slot0);
-            } else {
-              tma_load_3d_pair(vtile + c * box * 128, &tm_v, bar, 64 * int(rank), u.kv_head, slot0);
+              uint8_t* dstp = which == 0 ? ktile + b * (64 * 128) : vtile;
+              *reinterpret_cast<int4*>(dstp + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
             }
           }
-          __syncwarp();
         }
-        if (!ok) break;
-        // The unit's last S MMAs have read Q: the next unit's Q may be loaded.
-        ok = __all_sync(0xffffffffu, wait_parity(q_free, (qk - 1) & 1u, abort, p.timeout_ns));
-        if (!ok) break;
+        fence_proxy_async_smem();
+        __syncwarp();
       }
+      const uint32_t bar = lead_kv_full0 + uint32_t(slot) * 8u;
+      if (lane == 0) mbar_arrive_expect_tx_cluster(bar, tma_bytes);
+      __syncwarp();
+      // One lane per page chunk: K chunks first, then V chunks.
+      const int nk = has_k ? kchunks : 0, nv = has_v ? vchunks : 0;
+      for (int e = lane; e < nk + nv; e += 32) {
+        const bool is_k = e < nk;
+        const int c = is_k ? e : e - nk;
+        const int box = is_k ? kbox : vbox;
+        const int kc = (is_k ? key0k : key0v) + c * box;
+        if (kc + box > u.kv_end) continue;
+        const int32_t page = __ldg(pt + kc / p.page_size);
+        const bool in_pool = uint32_t(page) < uint32_t(p.num_pages);
+        bad_page |= !in_pool;
+        const int32_t slot0 = (in_pool ? page : p.num_pages) * p.page_size + kc % p.page_size;
+        if (is_k) {
+          for (int b = 0; b < 2; ++b)
+            tma_load_3d_pair(ktile + b * (64 * 128) + c * box * 128, &tm_k, bar, b * 64, u.kv_head, slot0);
+        } else {
+          tma_load_3d_pair(vtile + c * box * 128, &tm_v, bar, 64 * int(rank), u.kv_head, slot0);
+        }
+      }
+      __syncwarp();
+    };
+    // Q of both sub-tiles of unit u (the previous unit's last S MMAs have read the old Q).
+    auto load_q = [&](const PairUnit& u) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx_cluster(lead_q_full, 2 * C::kQBytes);
+        for (int i = 0; i < 2; ++i)
+          for (int b = 0; b < 2; ++b)
+            tma_load_3d_pair(smem + C::kQOff + i * C::kQBytes + b * C::kBoxBytes, &tm_q, lead_q_full, b * 64,
+                             u.st[i].head, int32_t(u.row_base + u.st[i].q0));
+      }
+      __syncwarp();
+    };
+    PairUnit u = pair_unit(p, vc0, rank);
+    const int32_t* pt = p.page_table + int64_t(u.hd.seq) * p.max_pages;
+    int t_next = 0;           // next stage of u to issue
+    bool ok = !__any_sync(0xffffffffu, *abort != 0);
+    if (ok) { load_q(u); ++qk; }
+    while (ok) {
+      // The rest of this unit's stages.
+      for (; t_next <= u.n; ++t_next, ++tg) {
+        const int slot = tg % C::kStages;
+        ok = __all_sync(0xffffffffu,
+                        wait_parity(&bars->kv_empty[slot], ((tg / C::kStages) & 1u) ^ 1u, abort, p.timeout_ns));
+        if (!ok) break;
+        issue_stage(u, pt, t_next, slot);
+      }
+      if (!ok) break;
       // The next unit: the leader reads the answer to the MMA thread's cancel
       // request and hands it on, the peer takes it from the ring.
       int nxt = -2;
@@ -890,7 +895,36 @@ attn_fwd_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           nxt = ring_take(bars, lead_unit_empty0, ring_k++, abort, p.timeout_ns);
         }
       }
-      vc = __shfl_sync(0xffffffffu, nxt, 0);
+      const int vn = __shfl_sync(0xffffffffu, nxt, 0);
+      if (vn < 0) break;
+      const PairUnit un = pair_unit(p, vn, rank);
+      const int32_t* pt_n = p.page_table + int64_t(un.hd.seq) * p.max_pages;
+      // While this unit's last S still reads Q, load the next unit's first
+      // K/V stages into the slots the MMA frees; then its Q.
+      int tn = 0;
+      const uint32_t qf_par = (qk - 1) & 1u;
+      const uint64_t t0 = global_timer_ns();
+      for (uint32_t it = 0; tn <= un.n; ++it) {
+        if (__shfl_sync(0xffffffffu, mbar_test_wait(q_free, qf_par) ? 1 : 0, 0)) break;
+        const int slot = tg % C::kStages;
+        if (__shfl_sync(0xffffffffu, mbar_test_wait(&bars->kv_empty[slot], ((tg / C::kStages) & 1u) ^ 1u) ? 1 : 0,
+                        0)) {
+          issue_stage(un, pt_n, tn, slot);
+          ++tn;
+          ++tg;
+          continue;
+        }
+        if ((it & 255u) == 255u &&
+            __shfl_sync(0xffffffffu, (*abort != 0 || global_timer_ns() - t0 > p.timeout_ns) ? 1 : 0, 0))
+          break;   // the blocking wait below gives up the same way
+      }
+      ok = __all_sync(0xffffffffu, wait_parity(q_free, qf_par, abort, p.timeout_ns));
+      if (!ok) break;
+      load_q(un);
+      ++qk;
+      u = un;
+      pt = pt_n;
+      t_next = tn;
     }
     if (bad_page && p.status) atomicOr(p.status, kStatusBadPage);
     // Copies of both CTAs land on the leader's barriers: the leader's producer

@@ -58,6 +58,26 @@ def test_bounded_wait_gives_up_and_context_stays_usable():
     _check_full(Run(Case(2, [200], 4, 2, 128, page_size=16)))
 
 
+def test_launch_after_a_timeout_aborts_at_entry():
+    """While the plan's status word carries a timeout from an earlier launch,
+    an attention launch (the persistent CTA-pair kernel here: several waves of
+    work units) gives up at entry in every cluster: it asks for no further
+    units, writes nothing and returns; after the status is read and cleared,
+    the same launch is exact again."""
+    run = Run(Case(4, [4096], 32, 4, 128, page_size=16))
+    ws = run.plan.workspace
+    status_off = ws.numel() - 256                      # the status word closes the workspace
+    ws[status_off:status_off + 4].copy_(torch.tensor([4, 0, 0, 0], dtype=torch.uint8))
+    with pytest.raises(zz.ZZError, match="outside the pool"):
+        run.plan.device_status()                       # the offset is the status word's
+    ws[status_off:status_off + 4].copy_(torch.tensor([1, 0, 0, 0], dtype=torch.uint8))
+    run.out.fill_(float("nan"))
+    run.attend()
+    assert torch.isnan(run.out.float()).all(), "an aborted launch wrote output"
+    assert run.plan.device_status() == 1               # timeout bit, read and cleared
+    _check_full(run)
+
+
 @pytest.mark.parametrize("case", [
     Case(2, [300, 517], 8, 2, 128, page_size=16, causal=False),
     Case(3, [700], 4, 4, 128, page_size=64, causal=False),              # row-pair mode

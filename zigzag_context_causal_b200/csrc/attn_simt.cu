@@ -3,7 +3,8 @@
 // one query head (small CTAs spread the short fp32 problems over many SMs);
 // four threads per query row, each owning D/4 of the head dimensions (partial
 // dot products combined with two shuffles); keys stream through shared memory
-// in chunks of 32 with an online (running max / running sum) softmax.  Same work list, half table and paged K/V addressing as the
+// in chunks of 32, the next chunk loaded into registers while the current one
+// is computed, with an online (running max / running sum) softmax.  Same work list, half table and paged K/V addressing as the
 // tensor-core kernel; the page "sgl-project--sglang/python/sglang/srt/layers/cp/zigzag.py",
 // run_attention, defines the per-half problem.
 #include <cuda_runtime.h>
@@ -82,26 +83,44 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtArgs a) {
   const int cta_last = a.causal ? hd.kv_pos0 + tile_last_row : hd.kv_full - 1;
   const int32_t* pt = a.page_table + int64_t(hd.seq) * a.max_pages;
   bool bad_page = false;   // a page outside the pool: its keys read as zeros, reported in status
-  for (int k0 = 0; k0 <= cta_last; k0 += kChunk) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < kChunk * D / 4; e += blockDim.x) {   // 16-byte pieces
-      const int j = e / (D / 4), x = (e % (D / 4)) * 4;
-      const int key = k0 + j;
-      float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), vx = kx;
+  // Each thread moves kPieces 16-byte pieces of K and of V per chunk.  The next
+  // chunk's pieces are loaded into registers while the current chunk is
+  // computed, so only the first chunk waits on memory (the page-table read and
+  // the K/V read it feeds are dependent loads).
+  constexpr int kPieces = kChunk * D / 4 / kSimtThreads;
+  static_assert(kPieces * kSimtThreads == kChunk * D / 4, "pieces per thread");
+  float4 kr[kPieces], vr[kPieces];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int it = 0; it < kPieces; ++it) {
+      const int e = threadIdx.x + it * kSimtThreads;
+      const int key = k0 + e / (D / 4), x = (e % (D / 4)) * 4;
+      kr[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+      vr[it] = kr[it];
       if (key < kv_end) {
         const int64_t slot = int64_t(pt[key / a.page_size]) * a.page_size + key % a.page_size;
         if (slot >= 0 && slot < a.num_slots) {
           const int64_t off = (slot * a.h_kv + kvh) * D + x;
-          kx = *reinterpret_cast<const float4*>(a.k_pool + off);
-          vx = *reinterpret_cast<const float4*>(a.v_pool + off);
+          kr[it] = *reinterpret_cast<const float4*>(a.k_pool + off);
+          vr[it] = *reinterpret_cast<const float4*>(a.v_pool + off);
         } else {
           bad_page = true;
         }
       }
-      *reinterpret_cast<float4*>(&ks[j][x]) = kx;
-      *reinterpret_cast<float4*>(&vs[j][x]) = vx;
+    }
+  };
+  fetch(0);
+  for (int k0 = 0; k0 <= cta_last; k0 += kChunk) {
+    __syncthreads();                       // the previous chunk is no longer read
+#pragma unroll
+    for (int it = 0; it < kPieces; ++it) {
+      const int e = threadIdx.x + it * kSimtThreads;
+      const int j = e / (D / 4), x = (e % (D / 4)) * 4;
+      *reinterpret_cast<float4*>(&ks[j][x]) = kr[it];
+      *reinterpret_cast<float4*>(&vs[j][x]) = vr[it];
     }
     __syncthreads();
+    if (k0 + kChunk <= cta_last) fetch(k0 + kChunk);
     float s[kChunk];
     float cmax = -CUDART_INF_F;
 #pragma unroll

@@ -299,7 +299,12 @@ zz_status_t zz_ipc_close(void* base);
  * bf16 runs the tcgen05/TMEM/TMA kernel (fp32 accumulate and softmax): for
  * d = 128 on pairs of CTAs (clusters of two that share each MMA; each CTA
  * loads half of every K and V tile), for d = 64 on single CTAs.  fp32 runs a
- * CUDA-core kernel in full fp32.
+ * CUDA-core kernel in full fp32.  The d = 128 kernel is persistent: a running
+ * cluster takes the work of clusters of the same launch that have not started
+ * (cluster launch control), so the work each cluster does varies from launch
+ * to launch, but every output row is computed by one cluster in a fixed order
+ * and the result is the same bit for bit.  Launches that share a plan on
+ * different streams may run at the same time (they share no device state).
  */
 zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_count,
                             const void* q, const void* k_pool, const void* v_pool,

@@ -304,7 +304,9 @@ zz_status_t zz_ipc_close(void* base);
  * (cluster launch control), so the work each cluster does varies from launch
  * to launch, but every output row is computed by one cluster in a fixed order
  * and the result is the same bit for bit.  Launches that share a plan on
- * different streams may run at the same time (they share no device state).
+ * different streams may run at the same time: they only read the plan's
+ * tables, and a status bit either of them sets lands in the plan's one
+ * status word.
  */
 zz_status_t zz_attn_prefill(const zz_plan_t* plan, int rank_begin, int rank_count,
                             const void* q, const void* k_pool, const void* v_pool,
